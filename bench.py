@@ -1,0 +1,385 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 MoBA prefill forward pass (one layer-forward = one step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step runs the whole path -- block mean-pool, gate/top-k, regrouping,
+history and own-block attention, merge -- on seeded synthetic inputs of the
+named workload (default: the scaling-law shape, batch 4 x 8192 tokens, 16
+heads, d=128, B=512, k=3, bf16). Inputs stay resident in HBM; they are larger
+than the 126 MB L2, so no flush is needed between steps.
+
+Metric: useful TFLOP/s (only QK^T and PV over the selected keys, 4*d per
+query-key pair), with ms per layer-forward beside it. Under torchrun every
+rank runs the same workload on its own GPU (weak scaling, no collective on
+the data path); `value` is the sum of all ranks' useful FLOPs divided by the
+slowest rank's time. Prints one JSON line on rank 0.
+
+--impl reference times the fp64 CPU oracle (the only reference this method
+has) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from moba_inputs import WORKLOADS, make_inputs, sample_rows  # noqa: E402
+
+METRIC = "moba_prefill_fwd_useful_tflops"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
+
+
+# ------------------------------------------------------------ accounting
+def flop_counts(w):
+    """(useful, history part, own-block part, dense causal) FLOPs of one layer-forward."""
+    useful = hist = cur = dense = 0
+    d, B, k, H = w.head_dim, w.block_size, w.topk, w.num_q_heads
+    for n in w.lengths:
+        p = np.arange(n, dtype=np.int64)
+        c = p // B
+        h = np.minimum(k - 1, c)
+        hist += int((4 * d * B * h).sum()) * H
+        cur += int((4 * d * (p - c * B + 1)).sum()) * H
+        dense += int((4 * d * (p + 1)).sum()) * H
+    useful = hist + cur
+    return useful, hist, cur, dense
+
+
+def row_flops(w, rows):
+    """Useful FLOPs of the sampled rows (row = t * Hq + h)."""
+    cu = np.concatenate([[0], np.cumsum(w.lengths)])
+    t = np.asarray(rows) // w.num_q_heads
+    b = np.searchsorted(cu, t, side="right") - 1
+    p = t - cu[b]
+    c = p // w.block_size
+    nkeys = np.minimum(w.topk - 1, c) * w.block_size + (p - c * w.block_size + 1)
+    return int((4 * w.head_dim * nkeys).sum())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def profile_traffic(kernel_src: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel; else None."""
+    path = os.path.join(ROOT, "profiles", f"attn_history_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    s = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    if not m or not s:
+        return None
+    sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+    return float(m.group(1)) if sha.startswith(s.group(1)) else None
+
+
+# ------------------------------------------------------------ clocks
+class ClockSampler:
+    def __init__(self, index: int):
+        self.proc = None
+        self.path = tempfile.mktemp(suffix=".csv")
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
+        os.unlink(self.path)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = max(mx, float(r[2]))
+                for nm, val in zip(names, r[5:9]):
+                    if val.strip().lower() == "active":
+                        reasons.add(nm)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ CPU oracle leg
+def time_oracle(w, q, k, v, cu, budget_s: float, seed: int = 7):
+    """Time the oracle on a bounded sample of rows; returns (tflops, rows, seconds, threads)."""
+    import oracle
+
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    total_rows = w.total_tokens * w.num_q_heads
+    n = 32
+    rows = sample_rows(total_rows, n, seed).numpy()
+    t0 = time.perf_counter()
+    oracle.forward_rows(qc, kc, vc, cu, w.block_size, w.topk, rows)
+    dt = time.perf_counter() - t0
+    n2 = int(min(total_rows, max(n, n * budget_s / max(dt, 1e-3))))
+    rows = sample_rows(total_rows, n2, seed + 1).numpy()
+    t0 = time.perf_counter()
+    oracle.forward_rows(qc, kc, vc, cu, w.block_size, w.topk, rows)
+    dt = time.perf_counter() - t0
+    return row_flops(w, rows) / dt / 1e12, len(rows), dt, oracle.num_threads()
+
+
+# ------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="scaling_8k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    useful, hist_flops, cur_flops, dense_flops = flop_counts(w)
+    config = {"workload": w.name, "batch": w.batch, "seq_lens": list(w.lengths),
+              "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+              "block_size": w.block_size, "topk": w.topk,
+              "l2": "inputs exceed L2 (q+k+v > 126 MB), no flush"}
+    dtype_name = "bf16" if w.dtype == torch.bfloat16 else "f32"
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        q, k, v, cu = make_inputs(w, "cpu")
+        per_step = []
+        t_all = time.perf_counter()
+        for _ in range(args.warmup + args.steps):
+            tf, nrows, dt, thr = time_oracle(w, q, k, v, cu, budget_s=2.0)
+            per_step.append((tf, nrows, dt))
+        per_step = per_step[args.warmup:]
+        tf = float(np.mean([x[0] for x in per_step]))
+        ms = float(np.mean([x[2] for x in per_step])) * 1e3
+        line = {"impl": "reference", "metric": METRIC, "value": tf, "unit": "TFLOP/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": {"kind": "oracle", "value": tf, "unit": "TFLOP/s", "cores": thr,
+                                 "sample": f"{per_step[0][1]} seeded (token, head) rows per step "
+                                           f"of {w.name}, useful FLOPs of those rows"},
+                "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import long_context_prefill_block_b200 as moba
+
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    q, k, v, cu = make_inputs(w, dev)
+    cu_d = cu.to(dev)
+    p = moba.make_params(q, k, cu, w.block_size, w.topk, w.max_seqlen)
+    ws = moba.workspace(p, dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+    L = moba.lib()
+    P = ctypes.byref(p)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+
+    def step():
+        rc = L.moba_forward(P, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                            ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(cu_d.data_ptr()),
+                            ctypes.c_void_p(out.data_ptr()), None, ctypes.c_void_p(ws.data_ptr()),
+                            ws.numel(), sp)
+        if rc:
+            raise RuntimeError(f"moba_forward failed: {rc}")
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    if moba.moba_device_status(dev) != 0:
+        raise RuntimeError("device status error after warm-up")
+
+    # ---- timed region: K steps, barrier + sync on both sides
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clock_info = clocks.stop() if clocks else None
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    value = useful * world / (ms * 1e-3) / 1e12
+
+    # ---- per-stage timing (same stream, CUDA events recorded by the library)
+    n_pass = L.moba_num_passes(P)
+    n_ev = 3 + 4 * n_pass
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    ev_arr = (ctypes.c_void_p * n_ev)(*[ctypes.c_void_p(e.cuda_event) for e in evs])
+    stage_ms = {"meanpool": 0.0, "gate_topk": 0.0, "regroup": 0.0, "attn_history": 0.0,
+                "attn_current": 0.0, "merge": 0.0}
+    reps = max(3, min(args.steps, 10))
+    for _ in range(reps):
+        rc = L.moba_forward_staged(P, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                   ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(cu_d.data_ptr()),
+                                   ctypes.c_void_p(out.data_ptr()), None,
+                                   ctypes.c_void_p(ws.data_ptr()), ws.numel(), ev_arr, n_ev, sp)
+        if rc:
+            raise RuntimeError(f"moba_forward_staged failed: {rc}")
+        torch.cuda.synchronize(dev)
+        stage_ms["meanpool"] += evs[0].elapsed_time(evs[1]) / reps
+        stage_ms["gate_topk"] += evs[1].elapsed_time(evs[2]) / reps
+        prev = evs[2]
+        for j in range(n_pass):
+            a, b_, c_, d_ = evs[3 + 4 * j: 7 + 4 * j]
+            stage_ms["regroup"] += prev.elapsed_time(a) / reps
+            stage_ms["attn_history"] += a.elapsed_time(b_) / reps
+            stage_ms["attn_current"] += b_.elapsed_time(c_) / reps
+            stage_ms["merge"] += c_.elapsed_time(d_) / reps
+            prev = d_
+
+    # ---- dense causal comparison at the same shape
+    dense_out = torch.empty_like(q)
+    for _ in range(2):
+        moba.dense_causal_forward(q, k, v, cu, max_seqlen=w.max_seqlen, out=dense_out)
+    torch.cuda.synchronize(dev)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dreps = 3
+    d0.record(stream)
+    for _ in range(dreps):
+        moba.dense_causal_forward(q, k, v, cu, max_seqlen=w.max_seqlen, out=dense_out)
+    d1.record(stream)
+    torch.cuda.synchronize(dev)
+    dense_ms = d0.elapsed_time(d1) / dreps
+    del dense_out
+
+    # ---- end to end through the public API with host buffers
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        rc = L.moba_forward(P, ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()),
+                            ctypes.c_void_p(dv.data_ptr()), ctypes.c_void_p(cu_d.data_ptr()),
+                            ctypes.c_void_p(out.data_ptr()), None, ctypes.c_void_p(ws.data_ptr()),
+                            ws.numel(), sp)
+        if rc:
+            raise RuntimeError(f"moba_forward failed: {rc}")
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    erep = max(3, min(args.steps, 10))
+    barrier()
+    e0.record(stream)
+    for _ in range(erep):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / erep)
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+    d2h = hout.numel() * hout.element_size()
+
+    peaks, peak_src = load_peaks()
+    hist_launch_ms = stage_ms["attn_history"] / n_pass
+    hist_launch_flops = hist_flops / n_pass
+    achieved = hist_launch_flops / (hist_launch_ms * 1e-3) / 1e12 if hist_launch_ms > 0 else 0.0
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    traffic = profile_traffic(os.path.join(ROOT, "long_context_prefill_block_b200", "csrc",
+                                           "attn_tc.cu"), w.name)
+    launches_per_step = 2 + 7 * n_pass
+
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        tf, nrows, dt, thr = time_oracle(w, q, k, v, cu, args.cpu_budget)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+               "sample": f"{nrows} seeded (token, head) rows of {w.name} ({dt:.1f} s), "
+                         "useful FLOPs of those rows"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype_name,
+        "data": "synthetic", "config": config,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "attn_history", "peak_source": f"{peak_src} bf16 burst"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": useful * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clock_info,
+        "stage_ms": stage_ms,
+        "useful_flop_per_step": useful,
+        "dense_causal_ms": dense_ms,
+        "speedup_vs_dense": dense_ms / ms,
+        "frac_of_peak_end_to_end": value / world / peak,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,159 @@
+/*
+ * moba.h -- C ABI of libmoba.so: the MoBA (Mixture of Block Attention)
+ * prefill forward pass on NVIDIA B200 (sm_100a).
+ *
+ * The method (PaperTrace knowledge page "2.1.3 MoBA", sections 1-3.1):
+ * keys are mean-pooled over contiguous blocks of B tokens (eq. 3); each
+ * query scores the blocks that lie wholly before its own block, always keeps
+ * its own block (which uses one of the k slots) and takes the k-1 best
+ * earlier blocks (section 2, section 2.1); exact softmax attention then runs
+ * over the raw keys and values of the chosen blocks, causal inside the own
+ * block (eq. 4-6), as ONE softmax over the union of candidates (eq. 7-8).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout: packed THD, row-major, contiguous, like flash-attn varlen:
+ *   q   [T, Hq,  d]     k, v [T, Hkv, d]     out [T, Hq, d]
+ *   cu_seqlens int32 [batch + 1], cu_seqlens[0] = 0, non-decreasing,
+ *   cu_seqlens[batch] = T; sequence b owns rows cu[b] .. cu[b+1]-1.
+ *   Blocks restart at every sequence start (block i of sequence b covers its
+ *   positions iB .. iB+B-1); no key crosses a sequence boundary.
+ * Heads: q head h reads kv head h / (Hq / Hkv) (grouped-query attention);
+ *   routing is done per q head.
+ * Element type: bf16 or fp32 (moba_params.dtype) for q, k, v and out;
+ *   arithmetic is fp32 (bf16 tensor-core products, fp32 accumulation).
+ * Pointers: every data pointer is a DEVICE pointer owned by the caller,
+ *   16-byte aligned. cu_seqlens is a device pointer too. The library never
+ *   allocates device memory, never frees, and never synchronises the stream;
+ *   temporary storage comes from the caller's workspace.
+ * Stream: `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ * Errors: arguments are validated on the host before anything is launched;
+ *   an invalid call returns a negative moba_status and launches nothing.
+ *   Errors found on the device (an index row that is not in canonical form,
+ *   a bounded wait that expired) are recorded in a per-device status word
+ *   read by moba_device_status().
+ */
+#ifndef MOBA_H_
+#define MOBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOBA_API __attribute__((visibility("default")))
+#else
+#define MOBA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOBA_OK = 0,
+  MOBA_ERR_INVALID_ARG = -1,  /* bad size, null pointer, misaligned pointer */
+  MOBA_ERR_UNSUPPORTED = -2,  /* valid but not implemented (d, dtype, k range) */
+  MOBA_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed */
+  MOBA_ERR_TIMEOUT = -4,      /* a bounded device wait expired */
+  MOBA_ERR_WORKSPACE = -5,    /* workspace null or smaller than moba_workspace_size() */
+  MOBA_ERR_BAD_INDICES = -6   /* an index row was not in canonical form */
+} moba_status;
+
+typedef enum { MOBA_BF16 = 0, MOBA_F32 = 1 } moba_dtype;
+
+typedef struct {
+  int batch;         /* number of sequences (>= 0) */
+  int total_tokens;  /* T = cu_seqlens[batch] */
+  int max_seqlen;    /* an upper bound on every sequence length */
+  int num_q_heads;   /* Hq */
+  int num_kv_heads;  /* Hkv; Hq % Hkv == 0 */
+  int head_dim;      /* d: 64 or 128 */
+  int block_size;    /* B >= 1 */
+  int topk;          /* k, 1 <= k <= 32; the current block uses one slot */
+  moba_dtype dtype;
+} moba_params;
+
+/* Number of key blocks reserved per sequence: ceil(max_seqlen / B). */
+MOBA_API int moba_num_blocks(const moba_params* p);
+
+/* Bytes of device workspace that moba_gate_topk, moba_forward and
+ * moba_forward_with_indices need for these parameters; 0 if the parameters
+ * are invalid. Partial results are kept for a group of kv heads at a time,
+ * so the size stays bounded for million-token inputs. */
+MOBA_API size_t moba_workspace_size(const moba_params* p);
+
+/* Block means, eq. (3): kbar[b][i][g][:] = mean of the keys of block i of
+ * sequence b and kv head g, over the positions present (a trailing partial
+ * block averages what it has). kbar: fp32 [batch][moba_num_blocks][Hkv][d];
+ * slots past a sequence's last block are written as 0. */
+MOBA_API moba_status moba_meanpool(const moba_params* p, const void* k, const int32_t* cu_seqlens,
+                          float* kbar, void* stream);
+
+/* The parameter-free gate with top-k (eq. 3 and section 2): for every token
+ * t and q head h, idx[t][h][:] = the chosen blocks of that query in
+ * ascending order -- the chosen earlier blocks first, then the query's own
+ * block c -- padded with -1 to k entries. Only blocks i < c are scored
+ * (s_i = q . kbar_i, fp32); blocks after c are never chosen; ties go to the
+ * lower block index. idx: int32 [T][Hq][k]. Uses the workspace for kbar. */
+MOBA_API moba_status moba_gate_topk(const moba_params* p, const void* q, const void* k,
+                           const int32_t* cu_seqlens, int32_t* idx, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* The full forward pass: gate, regrouping of queries by the block they
+ * chose, exact attention over the chosen history blocks (non-causal, eq. 6)
+ * and the own block (causal, eq. 5), merged by online softmax (eq. 7-8)
+ * into out [T][Hq][d] (input dtype). lse, if not NULL, receives the natural
+ * log-sum-exp of the scaled logits per (t, h), fp32 [T][Hq]. */
+MOBA_API moba_status moba_forward(const moba_params* p, const void* q, const void* k, const void* v,
+                         const int32_t* cu_seqlens, void* out, float* lse, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/* Number of passes over groups of kv heads that moba_forward makes. */
+MOBA_API int moba_num_passes(const moba_params* p);
+
+/* moba_forward with per-stage timing, the fair per-stage report of section
+ * 5.4 (gate, top-k, work-list build, sparse attention): `events` holds
+ * n_events >= 3 + 4 * moba_num_passes(p) cudaEvent_t handles (created by the
+ * caller, passed as void*). events[0] is recorded before the first launch,
+ * events[1] after the mean-pool, events[2] after the gate/top-k, and for pass
+ * j events[3+4j], [4+4j], [5+4j], [6+4j] after the regrouping, the history
+ * attention, the own-block attention and the merge. Results are identical to
+ * moba_forward. */
+MOBA_API moba_status moba_forward_staged(const moba_params* p, const void* q, const void* k,
+                                         const void* v, const int32_t* cu_seqlens, void* out,
+                                         float* lse, void* ws, size_t ws_bytes,
+                                         void* const* events, int n_events, void* stream);
+
+/* As moba_forward, with the chosen blocks supplied by the caller instead of
+ * the gate (forced candidates; a sliding-window or sink pattern is a special
+ * gate, section 3). idx: int32 [T][Hq][k] in the canonical form that
+ * moba_gate_topk writes: strictly ascending earlier blocks (each < c), then
+ * c, then -1. A row not in that form records MOBA_ERR_BAD_INDICES in the
+ * device status word; its output is then unspecified, but every access stays
+ * in bounds. */
+MOBA_API moba_status moba_forward_with_indices(const moba_params* p, const void* q, const void* k,
+                                      const void* v, const int32_t* cu_seqlens,
+                                      const int32_t* idx, void* out, float* lse, void* ws,
+                                      size_t ws_bytes, void* stream);
+
+/* Dense causal softmax attention, eq. (1) with a causal mask (every key
+ * j <= p of the query's own sequence), for comparison and for the full
+ * budget limit (section 4). block_size and topk in p must be valid but do
+ * not change the result. Needs no workspace. */
+MOBA_API moba_status dense_causal_forward(const moba_params* p, const void* q, const void* k,
+                                 const void* v, const int32_t* cu_seqlens, void* out, float* lse,
+                                 void* stream);
+
+/* Synchronises `stream`, returns the device status word of the current
+ * device (MOBA_OK, MOBA_ERR_TIMEOUT or MOBA_ERR_BAD_INDICES) and clears it
+ * if `clear` is non-zero. */
+MOBA_API moba_status moba_device_status(void* stream, int clear);
+
+/* Static description of a status code. */
+MOBA_API const char* moba_status_string(moba_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOBA_H_ */

@@ -1,0 +1,203 @@
+"""Python binding of libmoba.so, the B200 MoBA prefill forward pass.
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+torch provides device memory and the current stream. The binding refuses to
+run if the compiled library is missing; there is no fallback of any kind.
+
+Functions mirror the C ABI of include/moba.h:
+    moba_meanpool, moba_gate_topk, moba_forward, moba_forward_with_indices,
+    dense_causal_forward, moba_workspace_size, moba_device_status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoba.so")
+
+MOBA_OK, MOBA_ERR_INVALID_ARG, MOBA_ERR_UNSUPPORTED, MOBA_ERR_CUDA = 0, -1, -2, -3
+MOBA_ERR_TIMEOUT, MOBA_ERR_WORKSPACE, MOBA_ERR_BAD_INDICES = -4, -5, -6
+MOBA_BF16, MOBA_F32 = 0, 1
+
+EXPORTS = ("moba_num_blocks", "moba_workspace_size", "moba_meanpool", "moba_gate_topk",
+           "moba_forward", "moba_forward_with_indices", "dense_causal_forward",
+           "moba_device_status", "moba_status_string")
+
+
+class MobaParams(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("total_tokens", ctypes.c_int),
+                ("max_seqlen", ctypes.c_int), ("num_q_heads", ctypes.c_int),
+                ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("block_size", ctypes.c_int), ("topk", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class MobaError(RuntimeError):
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn}: {msg} (status {code})")
+        self.code = code
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmoba.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libmoba.so not built at {LIB_PATH}; run "
+                              "`python -m long_context_prefill_block_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, V, Z = ctypes.POINTER(MobaParams), ctypes.c_void_p, ctypes.c_size_t
+        L.moba_num_blocks.argtypes = [P]
+        L.moba_num_blocks.restype = ctypes.c_int
+        L.moba_workspace_size.argtypes = [P]
+        L.moba_workspace_size.restype = Z
+        L.moba_meanpool.argtypes = [P, V, V, V, V]
+        L.moba_gate_topk.argtypes = [P, V, V, V, V, V, Z, V]
+        L.moba_forward.argtypes = [P, V, V, V, V, V, V, V, Z, V]
+        L.moba_forward_with_indices.argtypes = [P, V, V, V, V, V, V, V, V, Z, V]
+        L.dense_causal_forward.argtypes = [P, V, V, V, V, V, V, V]
+        L.moba_device_status.argtypes = [V, ctypes.c_int]
+        L.moba_status_string.argtypes = [ctypes.c_int]
+        L.moba_status_string.restype = ctypes.c_char_p
+        for name in ("moba_meanpool", "moba_gate_topk", "moba_forward",
+                     "moba_forward_with_indices", "dense_causal_forward", "moba_device_status"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, code: int) -> None:
+    if code != MOBA_OK:
+        raise MobaError(fn, code, lib().moba_status_string(code).decode())
+
+
+def make_params(q: torch.Tensor, k: torch.Tensor, cu_seqlens: torch.Tensor, block_size: int,
+                topk: int, max_seqlen: Optional[int] = None) -> MobaParams:
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    batch = cu_seqlens.numel() - 1
+    if max_seqlen is None:
+        cu = cu_seqlens.detach().to("cpu", torch.int64)
+        max_seqlen = int((cu[1:] - cu[:-1]).max()) if batch > 0 else 0
+    if q.dtype == torch.bfloat16:
+        dt = MOBA_BF16
+    elif q.dtype == torch.float32:
+        dt = MOBA_F32
+    else:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    return MobaParams(batch, T, max_seqlen, Hq, Hkv, d, block_size, topk, dt)
+
+
+def _ptr(x: Optional[torch.Tensor]):
+    return None if x is None else ctypes.c_void_p(x.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dev_i32(cu: torch.Tensor, device) -> torch.Tensor:
+    return cu.to(device=device, dtype=torch.int32).contiguous()
+
+
+def _check_inputs(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def moba_workspace_size(params: MobaParams) -> int:
+    return int(lib().moba_workspace_size(ctypes.byref(params)))
+
+
+def moba_num_blocks(params: MobaParams) -> int:
+    return int(lib().moba_num_blocks(ctypes.byref(params)))
+
+
+def workspace(params: MobaParams, device) -> torch.Tensor:
+    return torch.empty(max(moba_workspace_size(params), 256), dtype=torch.uint8, device=device)
+
+
+def moba_meanpool(k: torch.Tensor, cu_seqlens: torch.Tensor, block_size: int,
+                  max_seqlen: Optional[int] = None) -> torch.Tensor:
+    """Block means fp32 [batch, num_blocks, Hkv, d]."""
+    _check_inputs(k)
+    p = make_params(k, k, cu_seqlens, block_size, 1, max_seqlen)
+    p.num_q_heads = p.num_kv_heads
+    cu = _dev_i32(cu_seqlens, k.device)
+    kbar = torch.empty((p.batch, moba_num_blocks(p), p.num_kv_heads, p.head_dim),
+                       dtype=torch.float32, device=k.device)
+    _check("moba_meanpool", lib().moba_meanpool(ctypes.byref(p), _ptr(k), _ptr(cu), _ptr(kbar),
+                                                _stream(k.device)))
+    return kbar
+
+
+def moba_gate_topk(q, k, cu_seqlens, block_size: int, topk: int, max_seqlen=None,
+                   ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Chosen blocks per (token, q head): int32 [T, Hq, topk], ascending, -1 padded."""
+    _check_inputs(q, k)
+    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen)
+    cu = _dev_i32(cu_seqlens, q.device)
+    ws = workspace(p, q.device) if ws is None else ws
+    idx = torch.empty((p.total_tokens, p.num_q_heads, topk), dtype=torch.int32, device=q.device)
+    _check("moba_gate_topk", lib().moba_gate_topk(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(cu),
+                                                  _ptr(idx), _ptr(ws), ws.numel(),
+                                                  _stream(q.device)))
+    return idx
+
+
+def moba_forward(q, k, v, cu_seqlens, block_size: int, topk: int, max_seqlen=None,
+                 return_lse: bool = False, ws: Optional[torch.Tensor] = None,
+                 out: Optional[torch.Tensor] = None):
+    """MoBA prefill forward: out [T, Hq, d] (input dtype) and optionally lse [T, Hq]."""
+    _check_inputs(q, k, v)
+    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen)
+    cu = _dev_i32(cu_seqlens, q.device)
+    ws = workspace(p, q.device) if ws is None else ws
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device) if return_lse else None
+    _check("moba_forward", lib().moba_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu),
+                                              _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                              _stream(q.device)))
+    return (out, lse) if return_lse else out
+
+
+def moba_forward_with_indices(q, k, v, cu_seqlens, idx, block_size: int, max_seqlen=None,
+                              return_lse: bool = False, ws: Optional[torch.Tensor] = None):
+    """MoBA forward with caller-chosen blocks idx int32 [T, Hq, topk] (canonical form)."""
+    _check_inputs(q, k, v, idx)
+    p = make_params(q, k, cu_seqlens, block_size, idx.shape[2], max_seqlen)
+    cu = _dev_i32(cu_seqlens, q.device)
+    ws = workspace(p, q.device) if ws is None else ws
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device) if return_lse else None
+    _check("moba_forward_with_indices",
+           lib().moba_forward_with_indices(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu),
+                                           _ptr(idx), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                           _stream(q.device)))
+    return (out, lse) if return_lse else out
+
+
+def dense_causal_forward(q, k, v, cu_seqlens, max_seqlen=None, return_lse: bool = False,
+                         out: Optional[torch.Tensor] = None):
+    """Dense causal attention over each sequence (the comparison kernel)."""
+    _check_inputs(q, k, v)
+    p = make_params(q, k, cu_seqlens, 128, 1, max_seqlen)
+    cu = _dev_i32(cu_seqlens, q.device)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device) if return_lse else None
+    _check("dense_causal_forward",
+           lib().dense_causal_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu),
+                                      _ptr(out), _ptr(lse), _stream(q.device)))
+    return (out, lse) if return_lse else out
+
+
+def moba_device_status(device=None, clear: bool = True) -> int:
+    """Synchronise the current stream and return (and clear) the device status word."""
+    return int(lib().moba_device_status(_stream(device), int(clear)))

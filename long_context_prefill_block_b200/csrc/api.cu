@@ -1,0 +1,326 @@
+// C ABI of libmoba.so (declared in include/moba.h): argument validation,
+// workspace layout and the launch sequence of the MoBA prefill forward pass
+// (PaperTrace "2.1.3 MoBA", section 3.1): mean-pool -> gate/top-k ->
+// regroup by key block -> history attention + own-block attention -> merge.
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "moba.h"
+
+namespace moba {
+// Per-device status word; kernels get its address, never the symbol.
+__device__ int g_status;
+
+cudaError_t launch_history_tc(const Dims& dm, const Chunk& ch, const void* q, const void* k,
+                              const void* v, const int32_t* cu, const Regroup& rg,
+                              const Partials& pt, int* status, cudaStream_t st);
+cudaError_t launch_current_tc(const Dims& dm, const Chunk& ch, const void* q, const void* k,
+                              const void* v, const int32_t* cu, const int32_t* idx,
+                              const Partials& pt, int* status, cudaStream_t st);
+cudaError_t launch_dense_tc(const Dims& dm, const void* q, const void* k, const void* v,
+                            const int32_t* cu, void* out, float* lse, int* status,
+                            cudaStream_t st);
+bool tc_supported(const Dims& dm);
+constexpr int kTcTileM = 128;
+}  // namespace moba
+
+using namespace moba;
+
+namespace {
+
+// Partial results are kept for at most this many bytes per pass; larger
+// problems are processed one group of kv heads at a time.
+constexpr size_t kPartialCap = size_t(32) << 30;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+moba_status validate(const moba_params* p, Dims& dm) {
+  if (!p) return MOBA_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->total_tokens < 0 || p->max_seqlen < 0 || p->num_q_heads <= 0 ||
+      p->num_kv_heads <= 0 || p->num_q_heads % p->num_kv_heads != 0 || p->block_size <= 0 ||
+      p->topk <= 0)
+    return MOBA_ERR_INVALID_ARG;
+  if (p->dtype != MOBA_BF16 && p->dtype != MOBA_F32) return MOBA_ERR_UNSUPPORTED;
+  if (p->head_dim != 64 && p->head_dim != 128) return MOBA_ERR_UNSUPPORTED;
+  if (p->topk > 32) return MOBA_ERR_UNSUPPORTED;
+  // int32 row ids: T * Hq * k must fit.
+  if ((int64_t)p->total_tokens * p->num_q_heads * p->topk >= (int64_t(1) << 31))
+    return MOBA_ERR_UNSUPPORTED;
+  dm.batch = p->batch;
+  dm.T = p->total_tokens;
+  dm.max_seqlen = p->max_seqlen;
+  dm.Hq = p->num_q_heads;
+  dm.Hkv = p->num_kv_heads;
+  dm.d = p->head_dim;
+  dm.B = p->block_size;
+  dm.topk = p->topk;
+  dm.nb = (int)(((int64_t)p->max_seqlen + p->block_size - 1) / p->block_size);
+  dm.dtype = p->dtype == MOBA_BF16 ? kBF16 : kF32;
+  return MOBA_OK;
+}
+
+bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; }
+
+struct Layout {
+  size_t kbar, idx, counts, cursor, list_off, tile_off, pairs, tiles, part_o, part_lse, total;
+  int ng;             // kv heads per pass
+  int64_t max_tiles;  // tile-table capacity per pass
+};
+
+// Workspace plan. `own_idx` reserves room for the index rows (moba_forward).
+Layout plan(const Dims& dm, bool own_idx) {
+  Layout L{};
+  const int grp = dm.Hq / dm.Hkv;
+  const size_t per_kv = (size_t)dm.T * grp * dm.topk * (dm.d * 4 + 4);
+  size_t ng = per_kv ? kPartialCap / per_kv : dm.Hkv;
+  if (ng < 1) ng = 1;
+  if (ng > (size_t)dm.Hkv) ng = dm.Hkv;
+  L.ng = (int)ng;
+  const int64_t n_lists = (int64_t)dm.batch * L.ng * dm.nb;
+  const int64_t max_pairs = (int64_t)dm.T * L.ng * grp * (dm.topk - 1);
+  const int tile_m = kSimtTileM < kTcTileM ? kSimtTileM : kTcTileM;
+  L.max_tiles = (max_pairs + tile_m - 1) / tile_m + n_lists;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L.kbar = take(sizeof(float) * (size_t)dm.batch * dm.nb * dm.Hkv * dm.d);
+  L.idx = take(own_idx ? sizeof(int32_t) * (size_t)dm.T * dm.Hq * dm.topk : 0);
+  L.counts = take(sizeof(int32_t) * n_lists);
+  L.cursor = take(sizeof(int32_t) * n_lists);
+  L.list_off = take(sizeof(int32_t) * (n_lists + 1));
+  L.tile_off = take(sizeof(int32_t) * (n_lists + 1));
+  L.pairs = take(sizeof(int32_t) * max_pairs);
+  L.tiles = take(sizeof(int2) * L.max_tiles);
+  L.part_o = take(sizeof(float) * (size_t)dm.T * L.ng * grp * dm.topk * dm.d);
+  L.part_lse = take(sizeof(float) * (size_t)dm.T * L.ng * grp * dm.topk);
+  L.total = off;
+  return L;
+}
+
+int* status_word() {
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) return nullptr;
+  return static_cast<int*>(ptr);
+}
+
+moba_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA; }
+
+#define MOBA_TRY(x)                                  \
+  do {                                               \
+    const cudaError_t e_ = (x);                      \
+    if (e_ != cudaSuccess) return MOBA_ERR_CUDA;     \
+  } while (0)
+
+int num_passes(const Dims& dm, const Layout& L) { return (dm.Hkv + L.ng - 1) / L.ng; }
+
+// Shared body of moba_forward, moba_forward_with_indices and
+// moba_forward_staged. With `events`, events[0] is recorded before the first
+// launch, events[1] after the mean-pool, events[2] after the gate, and for
+// pass j events[3+4j .. 6+4j] after regroup, history attention, own-block
+// attention and merge.
+moba_status forward_impl(const moba_params* p, const void* q, const void* k, const void* v,
+                         const int32_t* cu, const int32_t* idx_in, void* out, float* lse,
+                         void* ws, size_t ws_bytes, void* stream, void* const* events = nullptr,
+                         int n_events = 0) {
+  Dims dm;
+  moba_status s = validate(p, dm);
+  if (s != MOBA_OK) return s;
+  if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
+  if (!q || !k || !v || !cu || !out) return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (lse && !aligned16(lse)))
+    return MOBA_ERR_INVALID_ARG;
+  const Layout L = plan(dm, idx_in == nullptr);
+  if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOBA_ERR_WORKSPACE;
+  if (events && n_events < 3 + 4 * num_passes(dm, L)) return MOBA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int ev = 0;
+  auto mark = [&]() -> cudaError_t {
+    if (!events) return cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(events[ev++]), st);
+  };
+  MOBA_TRY(mark());
+  int* status = status_word();
+  if (!status) return MOBA_ERR_CUDA;
+  char* base = static_cast<char*>(ws);
+  float* kbar = reinterpret_cast<float*>(base + L.kbar);
+  const int32_t* idx = idx_in;
+  if (!idx_in) {
+    int32_t* own = reinterpret_cast<int32_t*>(base + L.idx);
+    MOBA_TRY(launch_meanpool(dm, k, cu, kbar, status, st));
+    MOBA_TRY(mark());
+    MOBA_TRY(launch_gate(dm, q, kbar, cu, own, status, st));
+    MOBA_TRY(mark());
+    idx = own;
+  } else {
+    MOBA_TRY(mark());
+    MOBA_TRY(mark());
+  }
+  const bool tc = tc_supported(dm);
+  const int grp = dm.Hq / dm.Hkv;
+  Regroup rg;
+  rg.counts = reinterpret_cast<int32_t*>(base + L.counts);
+  rg.cursor = reinterpret_cast<int32_t*>(base + L.cursor);
+  rg.list_off = reinterpret_cast<int32_t*>(base + L.list_off);
+  rg.tile_off = reinterpret_cast<int32_t*>(base + L.tile_off);
+  rg.pairs = reinterpret_cast<int32_t*>(base + L.pairs);
+  rg.tiles = reinterpret_cast<int2*>(base + L.tiles);
+  Partials pt{reinterpret_cast<float*>(base + L.part_o), reinterpret_cast<float*>(base + L.part_lse)};
+  for (int g0 = 0; g0 < dm.Hkv; g0 += L.ng) {
+    Chunk ch;
+    ch.g0 = g0;
+    ch.ng = dm.Hkv - g0 < L.ng ? dm.Hkv - g0 : L.ng;
+    ch.h0 = g0 * grp;
+    ch.nq = ch.ng * grp;
+    ch.n_lists = dm.batch * ch.ng * dm.nb;
+    ch.tile_m = tc ? kTcTileM : kSimtTileM;
+    const int64_t pairs = (int64_t)dm.T * ch.nq * (dm.topk - 1);
+    rg.max_tiles = (pairs + ch.tile_m - 1) / ch.tile_m + ch.n_lists;
+    MOBA_TRY(launch_regroup(dm, ch, idx, cu, rg, status, st));
+    MOBA_TRY(mark());
+    if (tc) {
+      MOBA_TRY(launch_history_tc(dm, ch, q, k, v, cu, rg, pt, status, st));
+      MOBA_TRY(mark());
+      MOBA_TRY(launch_current_tc(dm, ch, q, k, v, cu, idx, pt, status, st));
+    } else {
+      MOBA_TRY(launch_history_simt(dm, ch, q, k, v, cu, rg, pt, st));
+      MOBA_TRY(mark());
+      MOBA_TRY(launch_current_simt(dm, ch, q, k, v, cu, idx, pt, st));
+    }
+    MOBA_TRY(mark());
+    MOBA_TRY(launch_merge(dm, ch, idx, cu, pt, out, lse, st));
+    MOBA_TRY(mark());
+  }
+  return MOBA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moba_num_blocks(const moba_params* p) {
+  Dims dm;
+  if (validate(p, dm) != MOBA_OK) return 0;
+  return dm.nb;
+}
+
+size_t moba_workspace_size(const moba_params* p) {
+  Dims dm;
+  if (validate(p, dm) != MOBA_OK) return 0;
+  return plan(dm, true).total;
+}
+
+moba_status moba_meanpool(const moba_params* p, const void* k, const int32_t* cu_seqlens,
+                          float* kbar, void* stream) {
+  Dims dm;
+  moba_status s = validate(p, dm);
+  if (s != MOBA_OK) return s;
+  if (dm.batch == 0 || dm.nb == 0) return MOBA_OK;
+  if (!k || !cu_seqlens || !kbar || !aligned16(k) || !aligned16(kbar)) return MOBA_ERR_INVALID_ARG;
+  int* status = status_word();
+  if (!status) return MOBA_ERR_CUDA;
+  return cuda_status(launch_meanpool(dm, k, cu_seqlens, kbar, status,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+moba_status moba_gate_topk(const moba_params* p, const void* q, const void* k,
+                           const int32_t* cu_seqlens, int32_t* idx, void* ws, size_t ws_bytes,
+                           void* stream) {
+  Dims dm;
+  moba_status s = validate(p, dm);
+  if (s != MOBA_OK) return s;
+  if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
+  if (!q || !k || !cu_seqlens || !idx || !aligned16(q) || !aligned16(k)) return MOBA_ERR_INVALID_ARG;
+  const Layout L = plan(dm, true);
+  if (!ws || ws_bytes < L.kbar + sizeof(float) * (size_t)dm.batch * dm.nb * dm.Hkv * dm.d ||
+      !aligned16(ws))
+    return MOBA_ERR_WORKSPACE;
+  int* status = status_word();
+  if (!status) return MOBA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* kbar = reinterpret_cast<float*>(static_cast<char*>(ws) + L.kbar);
+  MOBA_TRY(launch_meanpool(dm, k, cu_seqlens, kbar, status, st));
+  MOBA_TRY(launch_gate(dm, q, kbar, cu_seqlens, idx, status, st));
+  return MOBA_OK;
+}
+
+moba_status moba_forward(const moba_params* p, const void* q, const void* k, const void* v,
+                         const int32_t* cu_seqlens, void* out, float* lse, void* ws,
+                         size_t ws_bytes, void* stream) {
+  return forward_impl(p, q, k, v, cu_seqlens, nullptr, out, lse, ws, ws_bytes, stream);
+}
+
+int moba_num_passes(const moba_params* p) {
+  Dims dm;
+  if (validate(p, dm) != MOBA_OK) return 0;
+  return num_passes(dm, plan(dm, true));
+}
+
+moba_status moba_forward_staged(const moba_params* p, const void* q, const void* k, const void* v,
+                                const int32_t* cu_seqlens, void* out, float* lse, void* ws,
+                                size_t ws_bytes, void* const* events, int n_events,
+                                void* stream) {
+  if (!events) return MOBA_ERR_INVALID_ARG;
+  return forward_impl(p, q, k, v, cu_seqlens, nullptr, out, lse, ws, ws_bytes, stream, events,
+                      n_events);
+}
+
+moba_status moba_forward_with_indices(const moba_params* p, const void* q, const void* k,
+                                      const void* v, const int32_t* cu_seqlens,
+                                      const int32_t* idx, void* out, float* lse, void* ws,
+                                      size_t ws_bytes, void* stream) {
+  Dims dm;
+  moba_status s = validate(p, dm);
+  if (s != MOBA_OK) return s;
+  if (dm.T > 0 && dm.batch > 0 && !idx) return MOBA_ERR_INVALID_ARG;
+  return forward_impl(p, q, k, v, cu_seqlens, idx, out, lse, ws, ws_bytes, stream);
+}
+
+moba_status dense_causal_forward(const moba_params* p, const void* q, const void* k,
+                                 const void* v, const int32_t* cu_seqlens, void* out, float* lse,
+                                 void* stream) {
+  Dims dm;
+  moba_status s = validate(p, dm);
+  if (s != MOBA_OK) return s;
+  if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
+  if (!q || !k || !v || !cu_seqlens || !out) return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (lse && !aligned16(lse)))
+    return MOBA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = status_word();
+  if (!status) return MOBA_ERR_CUDA;
+  if (tc_supported(dm)) return cuda_status(launch_dense_tc(dm, q, k, v, cu_seqlens, out, lse, status, st));
+  return cuda_status(launch_dense_simt(dm, q, k, v, cu_seqlens, out, lse, st));
+}
+
+moba_status moba_device_status(void* stream, int clear) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOBA_ERR_CUDA;
+  int value = 0;
+  if (cudaMemcpyFromSymbol(&value, g_status, sizeof(int)) != cudaSuccess) return MOBA_ERR_CUDA;
+  if (clear) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return MOBA_ERR_CUDA;
+  }
+  return static_cast<moba_status>(value);
+}
+
+const char* moba_status_string(moba_status s) {
+  switch (s) {
+    case MOBA_OK: return "ok";
+    case MOBA_ERR_INVALID_ARG: return "invalid argument";
+    case MOBA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOBA_ERR_CUDA: return "CUDA error";
+    case MOBA_ERR_TIMEOUT: return "bounded device wait expired";
+    case MOBA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOBA_ERR_BAD_INDICES: return "index row not in canonical form";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

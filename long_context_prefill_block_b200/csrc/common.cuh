@@ -1,0 +1,139 @@
+// Shared device helpers and the launch interface between the C ABI (api.cu)
+// and the kernels. Nothing here is visible outside libmoba.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moba {
+
+constexpr int kBF16 = 0;
+constexpr int kF32 = 1;
+
+// Device status codes (same values as moba_status).
+constexpr int kStInvalidArg = -1;
+constexpr int kStTimeout = -4;
+constexpr int kStBadIndices = -6;
+
+// Sizes of one call, validated on the host.
+struct Dims {
+  int batch;       // sequences
+  int T;           // total tokens
+  int max_seqlen;  // bound on every sequence length
+  int Hq, Hkv;     // heads
+  int d;           // head dim
+  int B;           // block size
+  int topk;        // k
+  int nb;          // blocks reserved per sequence = ceil(max_seqlen / B)
+  int dtype;       // kBF16 / kF32
+};
+
+// Work of one pass over a group of kv heads [g0, g0 + ng): its q heads are
+// [g0 * grp, (g0 + ng) * grp). Partial results are indexed by
+// prow = ((t * nq) + h_local) * topk + slot, nq = ng * grp.
+struct Chunk {
+  int g0, ng;      // kv heads of this pass
+  int h0, nq;      // q heads of this pass
+  int n_lists;     // batch * ng * nb regroup lists
+  int tile_m;      // query rows per history tile
+};
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// 16-byte vector of elements widened to fp32.
+template <typename T>
+struct Vec16;
+template <>
+struct Vec16<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void load(const float* p, float* out) {
+    const float4 r = __ldg(reinterpret_cast<const float4*>(p));
+    out[0] = r.x; out[1] = r.y; out[2] = r.z; out[3] = r.w;
+  }
+};
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float* out) {
+    const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      out[2 * i] = __uint_as_float(w[i] << 16);
+      out[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+};
+
+// First error wins.
+__device__ __forceinline__ void set_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// Sequence bounds with a device-side check against max_seqlen.
+__device__ __forceinline__ bool seq_bounds(const Dims& dm, const int32_t* cu, int b, int64_t& start,
+                                           int& len, int* status) {
+  start = cu[b];
+  len = cu[b + 1] - cu[b];
+  if (len < 0 || len > dm.max_seqlen) {
+    set_status(status, kStInvalidArg);
+    return false;
+  }
+  return true;
+}
+
+}  // namespace moba
+
+// ---- launchers (host), one per kernel family -------------------------------
+namespace moba {
+
+cudaError_t launch_meanpool(const Dims& dm, const void* k, const int32_t* cu, float* kbar,
+                            int* status, cudaStream_t st);
+cudaError_t launch_gate(const Dims& dm, const void* q, const float* kbar, const int32_t* cu,
+                        int32_t* idx, int* status, cudaStream_t st);
+
+// Regrouping of (query, head, slot) by the history block it chose.
+struct Regroup {
+  int32_t* counts;     // [n_lists]
+  int32_t* cursor;     // [n_lists]
+  int32_t* list_off;   // [n_lists + 1]
+  int32_t* tile_off;   // [n_lists + 1]; tile_off[n_lists] = number of tiles
+  int32_t* pairs;      // [max pairs] partial-row ids grouped by list
+  int2* tiles;         // [max tiles] (list, first row in list)
+  int64_t max_tiles;
+};
+cudaError_t launch_regroup(const Dims& dm, const Chunk& ch, const int32_t* idx, const int32_t* cu,
+                           const Regroup& rg, int* status, cudaStream_t st);
+
+// Partial attention results of one pass.
+struct Partials {
+  float* o;    // [T * nq * topk][d], normalised
+  float* lse;  // [T * nq * topk]
+};
+
+// Portable SIMT kernels (fp32 or bf16 inputs, any block size).
+cudaError_t launch_history_simt(const Dims& dm, const Chunk& ch, const void* q, const void* k,
+                                const void* v, const int32_t* cu, const Regroup& rg,
+                                const Partials& pt, cudaStream_t st);
+cudaError_t launch_current_simt(const Dims& dm, const Chunk& ch, const void* q, const void* k,
+                                const void* v, const int32_t* cu, const int32_t* idx,
+                                const Partials& pt, cudaStream_t st);
+cudaError_t launch_dense_simt(const Dims& dm, const void* q, const void* k, const void* v,
+                              const int32_t* cu, void* out, float* lse, cudaStream_t st);
+constexpr int kSimtTileM = 32;
+
+cudaError_t launch_merge(const Dims& dm, const Chunk& ch, const int32_t* idx, const int32_t* cu,
+                         const Partials& pt, void* out, float* lse, cudaStream_t st);
+
+}  // namespace moba

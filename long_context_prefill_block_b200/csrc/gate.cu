@@ -1,0 +1,208 @@
+// The parameter-free MoBA gate with causal block mask, forced own block and
+// top-k (PaperTrace "2.1.3 MoBA", section 1 eq. 3, section 2, section 2.1):
+//   s_i = q . kbar_i for the blocks i < c wholly before the query's block c;
+//   blocks after c are never chosen and the full mean of block c (which
+//   would include future keys) is never scored; block c is always chosen and
+//   uses one of the k slots; the other min(k-1, c) slots take the highest
+//   s_i, equal scores going to the lower block index.
+//
+// Scores are fp32 FMA (q widened from bf16, kbar fp32): the near-tie band of
+// the parity check is 1e-4 relative and bf16/tf32 products would flip far
+// more ranks than that. One CTA scores 32 queries of one (sequence, head);
+// 4 threads per query each scan a quarter of every 32-block chunk of kbar
+// held in shared memory and keep a sorted register list of their best
+// KM >= k-1 blocks; the four lists are merged by warp shuffles.
+#include <climits>
+#include <cmath>
+
+#include "common.cuh"
+
+namespace moba {
+namespace {
+
+constexpr int kQ = 32;        // queries per CTA
+constexpr int kThreads = 128; // 4 threads per query
+constexpr int kCh = 32;       // kbar rows per shared-memory chunk
+
+__device__ __forceinline__ bool better(float s, int i, float t, int j) {
+  return s > t || (s == t && i < j);
+}
+
+template <int KM>
+__device__ __forceinline__ void insert(float (&ts)[KM], int (&ti)[KM], float s, int i) {
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    if (better(s, i, ts[j], ti[j])) {
+      const float fs = ts[j];
+      const int fi = ti[j];
+      ts[j] = s;
+      ti[j] = i;
+      s = fs;
+      i = fi;
+    }
+  }
+}
+
+template <typename T, int D, int KM>
+__global__ void __launch_bounds__(kThreads) gate_kernel(Dims dm, const T* __restrict__ q,
+                                                        const float* __restrict__ kbar,
+                                                        const int32_t* __restrict__ cu,
+                                                        int32_t* __restrict__ idx, int* status) {
+  __shared__ __align__(16) float qs[kQ][D + 4];
+  __shared__ __align__(16) float kb[kCh][D + 4];
+
+  const int b = blockIdx.y, h = blockIdx.z;
+  const int g = h / (dm.Hq / dm.Hkv);
+  int64_t start;
+  int len;
+  if (!seq_bounds(dm, cu, b, start, len, status)) return;
+  const int p0 = blockIdx.x * kQ;
+  if (p0 >= len) return;
+
+  constexpr int VEC = Vec16<T>::N, TPR = D / VEC;
+  for (int e = threadIdx.x; e < kQ * TPR; e += kThreads) {
+    const int r = e / TPR, l = e % TPR;
+    float x[VEC];
+    if (p0 + r < len) {
+      Vec16<T>::load(q + ((start + p0 + r) * dm.Hq + h) * (int64_t)D + l * VEC, x);
+    } else {
+#pragma unroll
+      for (int u = 0; u < VEC; ++u) x[u] = 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < VEC; ++u) qs[r][l * VEC + u] = x[u];
+  }
+
+  const int qi = threadIdx.x >> 2, part = threadIdx.x & 3;
+  const int p = p0 + qi;
+  const bool valid = p < len;
+  const int c = valid ? p / dm.B : 0;
+  const int cmax = (min(p0 + kQ, len) - 1) / dm.B;  // blocks any query of the tile may score
+
+  float ts[KM];
+  int ti[KM];
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    ts[j] = -INFINITY;
+    ti[j] = INT_MAX;
+  }
+
+  for (int base = 0; base < cmax; base += kCh) {
+    __syncthreads();
+    const int nblk = min(kCh, cmax - base);
+    for (int e = threadIdx.x; e < nblk * (D / 4); e += kThreads) {
+      const int r = e / (D / 4), l = e % (D / 4);
+      *reinterpret_cast<float4*>(&kb[r][l * 4]) = __ldg(reinterpret_cast<const float4*>(
+          kbar + (((int64_t)b * dm.nb + base + r) * dm.Hkv + g) * D + l * 4));
+    }
+    __syncthreads();
+    float s[kCh / 4];
+#pragma unroll
+    for (int u = 0; u < kCh / 4; ++u) s[u] = 0.f;
+    const float4* qa = reinterpret_cast<const float4*>(qs[qi]);
+#pragma unroll 4
+    for (int x4 = 0; x4 < D / 4; ++x4) {
+      const float4 a = qa[x4];
+#pragma unroll
+      for (int u = 0; u < kCh / 4; ++u) {
+        const float4 w = reinterpret_cast<const float4*>(kb[part + 4 * u])[x4];
+        s[u] = fmaf(a.x, w.x, s[u]);
+        s[u] = fmaf(a.y, w.y, s[u]);
+        s[u] = fmaf(a.z, w.z, s[u]);
+        s[u] = fmaf(a.w, w.w, s[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kCh / 4; ++u) {
+      const int jj = part + 4 * u;
+      const int i = base + jj;
+      if (jj < nblk && i < c) insert<KM>(ts, ti, s[u], i);
+    }
+  }
+
+  // Merge the four lists of each query: round r takes the best head.
+  const int hsel = valid ? min(dm.topk - 1, c) : 0;
+  int sel[KM];
+#pragma unroll
+  for (int r = 0; r < KM; ++r) {
+    sel[r] = INT_MAX;
+    if (r < dm.topk - 1) {
+      float bs = ts[0];
+      int bi = ti[0], owner = part;
+#pragma unroll
+      for (int off = 1; off <= 2; off <<= 1) {
+        const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        const int oo = __shfl_xor_sync(0xffffffffu, owner, off);
+        if (better(os, oi, bs, bi)) {
+          bs = os;
+          bi = oi;
+          owner = oo;
+        }
+      }
+      if (owner == part) {
+#pragma unroll
+        for (int j = 0; j + 1 < KM; ++j) {
+          ts[j] = ts[j + 1];
+          ti[j] = ti[j + 1];
+        }
+        ts[KM - 1] = -INFINITY;
+        ti[KM - 1] = INT_MAX;
+      }
+      if (r < hsel) sel[r] = bi;
+    }
+  }
+  if (part != 0 || !valid) return;
+  // ascending order of the chosen earlier blocks
+#pragma unroll
+  for (int a = 0; a < KM; ++a) {
+#pragma unroll
+    for (int j = 0; j + 1 < KM - a; ++j) {
+      if (sel[j] > sel[j + 1]) {
+        const int x = sel[j];
+        sel[j] = sel[j + 1];
+        sel[j + 1] = x;
+      }
+    }
+  }
+  int32_t* row = idx + ((start + p) * dm.Hq + h) * (int64_t)dm.topk;
+#pragma unroll
+  for (int r = 0; r <= KM; ++r) {
+    if (r < dm.topk) row[r] = r < hsel ? sel[r < KM ? r : KM - 1] : (r == hsel ? c : -1);
+  }
+}
+
+template <typename T, int D, int KM>
+cudaError_t run(const Dims& dm, const void* q, const float* kbar, const int32_t* cu, int32_t* idx,
+                int* status, cudaStream_t st) {
+  dim3 grid((dm.max_seqlen + kQ - 1) / kQ, dm.batch, dm.Hq);
+  gate_kernel<T, D, KM><<<grid, kThreads, 0, st>>>(dm, static_cast<const T*>(q), kbar, cu, idx,
+                                                   status);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t by_k(const Dims& dm, const void* q, const float* kbar, const int32_t* cu, int32_t* idx,
+                 int* status, cudaStream_t st) {
+  const int need = dm.topk - 1;
+  if (need <= 1) return run<T, D, 1>(dm, q, kbar, cu, idx, status, st);
+  if (need <= 2) return run<T, D, 2>(dm, q, kbar, cu, idx, status, st);
+  if (need <= 4) return run<T, D, 4>(dm, q, kbar, cu, idx, status, st);
+  if (need <= 8) return run<T, D, 8>(dm, q, kbar, cu, idx, status, st);
+  if (need <= 16) return run<T, D, 16>(dm, q, kbar, cu, idx, status, st);
+  return run<T, D, 32>(dm, q, kbar, cu, idx, status, st);
+}
+
+}  // namespace
+
+cudaError_t launch_gate(const Dims& dm, const void* q, const float* kbar, const int32_t* cu,
+                        int32_t* idx, int* status, cudaStream_t st) {
+  if (dm.batch == 0 || dm.max_seqlen == 0) return cudaSuccess;
+  if (dm.dtype == kBF16)
+    return dm.d == 128 ? by_k<__nv_bfloat16, 128>(dm, q, kbar, cu, idx, status, st)
+                       : by_k<__nv_bfloat16, 64>(dm, q, kbar, cu, idx, status, st);
+  return dm.d == 128 ? by_k<float, 128>(dm, q, kbar, cu, idx, status, st)
+                     : by_k<float, 64>(dm, q, kbar, cu, idx, status, st);
+}
+
+}  // namespace moba

@@ -1,0 +1,76 @@
+// Block mean-pooling of keys (PaperTrace "2.1.3 MoBA", section 1, eq. 3):
+// kbar_i = (1/B) * sum of the raw keys of block i, one routing vector per
+// (sequence, block, kv head), fp32.
+//
+// One CTA per (block, sequence, kv head). Each thread owns 16 bytes of a key
+// row (8 bf16 or 4 fp32 elements); a row is read by D*size/16 consecutive
+// threads, so every warp load is contiguous 128-256 B. Rows of one block are
+// spread over the CTA's row groups, summed in registers and reduced once in
+// shared memory: K is read exactly once (HBM-bound).
+#include "common.cuh"
+
+namespace moba {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads) meanpool_kernel(Dims dm, const T* __restrict__ k,
+                                                            const int32_t* __restrict__ cu,
+                                                            float* __restrict__ kbar,
+                                                            int* status) {
+  constexpr int VEC = Vec16<T>::N;   // elements per 16-byte load
+  constexpr int TPR = D / VEC;       // threads per key row
+  constexpr int RG = kThreads / TPR; // rows in flight
+  __shared__ float red[RG][D + 1];
+
+  const int i = blockIdx.x, b = blockIdx.y, g = blockIdx.z;
+  int64_t start;
+  int len;
+  const bool ok = seq_bounds(dm, cu, b, start, len, status);
+  const int j0 = i * dm.B;
+  const int j1 = ok ? min(len, j0 + dm.B) : j0;
+  const int lane = threadIdx.x % TPR, rg = threadIdx.x / TPR;
+
+  float acc[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+  for (int j = j0 + rg; j < j1; j += RG) {
+    float x[VEC];
+    Vec16<T>::load(k + ((start + j) * dm.Hkv + g) * (int64_t)D + lane * VEC, x);
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] += x[e];
+  }
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) red[rg][lane * VEC + e] = acc[e];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float s = 0.f;
+#pragma unroll 8
+    for (int r = 0; r < RG; ++r) s += red[r][threadIdx.x];
+    const int n = j1 - j0;
+    kbar[(((int64_t)b * dm.nb + i) * dm.Hkv + g) * D + threadIdx.x] = n > 0 ? s / (float)n : 0.f;
+  }
+}
+
+template <typename T, int D>
+cudaError_t run(const Dims& dm, const void* k, const int32_t* cu, float* kbar, int* status,
+                cudaStream_t st) {
+  dim3 grid(dm.nb, dm.batch, dm.Hkv);
+  meanpool_kernel<T, D><<<grid, kThreads, 0, st>>>(dm, static_cast<const T*>(k), cu, kbar, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_meanpool(const Dims& dm, const void* k, const int32_t* cu, float* kbar,
+                            int* status, cudaStream_t st) {
+  if (dm.batch == 0 || dm.nb == 0) return cudaSuccess;
+  if (dm.dtype == kBF16)
+    return dm.d == 128 ? run<__nv_bfloat16, 128>(dm, k, cu, kbar, status, st)
+                       : run<__nv_bfloat16, 64>(dm, k, cu, kbar, status, st);
+  return dm.d == 128 ? run<float, 128>(dm, k, cu, kbar, status, st)
+                     : run<float, 64>(dm, k, cu, kbar, status, st);
+}
+
+}  // namespace moba

@@ -1,0 +1,178 @@
+// Regrouping of queries by the key block they chose (PaperTrace "2.1.3
+// MoBA", section 3.1 steps 3 and 5, section 5.4): the query -> block choices
+// are inverted into one list per (sequence, kv head, history block) of the
+// (query, q head, slot) entries that read it, so that one contiguous K/V
+// block serves a dense tile of queries -- the MoE token-dispatch pattern of
+// histogram, exclusive scan and scatter.
+//
+// An entry is a partial-row id prow = ((t * nq) + h_local) * k + slot, where
+// slot is the entry's position in the query's index row; the history kernel
+// writes its partial result there and the merge reads it back in query
+// order, which also restores the original order. Entries inside a list are
+// in atomic-arrival order: each query's result depends only on its own row,
+// so the order changes no output bit.
+//
+// The count pass also checks each index row's canonical form (strictly
+// ascending earlier blocks, then the own block c, then -1 padding) and
+// records kStBadIndices for a row that breaks it; such entries are skipped.
+#include "common.cuh"
+
+namespace moba {
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kScanThreads = 1024;
+
+// Walks one index row; calls f(slot, block) for every history entry and
+// returns false if the row is not canonical.
+template <typename F>
+__device__ __forceinline__ bool walk_row(const int32_t* row, int topk, int c, F f) {
+  int prev = -1;
+  bool seen_c = false, ok = true;
+  for (int r = 0; r < topk; ++r) {
+    const int e = row[r];
+    if (seen_c) {
+      ok &= (e == -1);
+    } else if (e == c) {
+      seen_c = true;
+    } else if (e >= 0 && e < c && e > prev) {
+      prev = e;
+      f(r, e);
+    } else {
+      ok = false;
+    }
+  }
+  return ok && seen_c;
+}
+
+template <bool SCATTER>
+__global__ void __launch_bounds__(kThreads) regroup_pass(Dims dm, Chunk ch,
+                                                         const int32_t* __restrict__ idx,
+                                                         const int32_t* __restrict__ cu,
+                                                         int32_t* counts, int32_t* cursor,
+                                                         const int32_t* __restrict__ list_off,
+                                                         int32_t* pairs, int* status) {
+  const int b = blockIdx.y, hl = blockIdx.z;
+  const int h = ch.h0 + hl;
+  const int grp = dm.Hq / dm.Hkv;
+  const int gl = h / grp - ch.g0;
+  int64_t start;
+  int len;
+  if (!seq_bounds(dm, cu, b, start, len, SCATTER ? nullptr : status)) return;
+  const int p = blockIdx.x * kThreads + threadIdx.x;
+  if (p >= len) return;
+  const int64_t t = start + p;
+  const int c = p / dm.B;
+  const int32_t* row = idx + (t * dm.Hq + h) * (int64_t)dm.topk;
+  const int list0 = (b * ch.ng + gl) * dm.nb;
+  const int64_t prow0 = (t * ch.nq + hl) * (int64_t)dm.topk;
+  const bool ok = walk_row(row, dm.topk, c, [&](int slot, int e) {
+    if (SCATTER) {
+      const int list = list0 + e;
+      const int pos = atomicAdd(&cursor[list], 1);
+      pairs[list_off[list] + pos] = (int32_t)(prow0 + slot);
+    } else {
+      atomicAdd(&counts[list0 + e], 1);
+    }
+  });
+  if (!SCATTER && !ok) set_status(status, kStBadIndices);
+}
+
+// Exclusive scans of the list sizes and of their tile counts (one CTA).
+__global__ void __launch_bounds__(kScanThreads) regroup_scan(int n_lists, int tile_m,
+                                                            const int32_t* __restrict__ counts,
+                                                            int32_t* list_off, int32_t* tile_off) {
+  __shared__ int warp_a[kScanThreads / 32], warp_b[kScanThreads / 32];
+  __shared__ int carry_a, carry_b;
+  if (threadIdx.x == 0) carry_a = carry_b = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int base = 0; base < n_lists; base += kScanThreads) {
+    const int i = base + threadIdx.x;
+    const int a = i < n_lists ? counts[i] : 0;
+    const int bt = (a + tile_m - 1) / tile_m;
+    int xa = a, xb = bt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int ya = __shfl_up_sync(0xffffffffu, xa, off);
+      const int yb = __shfl_up_sync(0xffffffffu, xb, off);
+      if (lane >= off) {
+        xa += ya;
+        xb += yb;
+      }
+    }
+    if (lane == 31) {
+      warp_a[wid] = xa;
+      warp_b[wid] = xb;
+    }
+    __syncthreads();
+    if (wid == 0) {
+      int va = warp_a[lane], vb = warp_b[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int ya = __shfl_up_sync(0xffffffffu, va, off);
+        const int yb = __shfl_up_sync(0xffffffffu, vb, off);
+        if (lane >= off) {
+          va += ya;
+          vb += yb;
+        }
+      }
+      warp_a[lane] = va;
+      warp_b[lane] = vb;
+    }
+    __syncthreads();
+    const int pa = (wid ? warp_a[wid - 1] : 0) + xa - a + carry_a;
+    const int pb = (wid ? warp_b[wid - 1] : 0) + xb - bt + carry_b;
+    if (i < n_lists) {
+      list_off[i] = pa;
+      tile_off[i] = pb;
+    }
+    __syncthreads();
+    if (threadIdx.x == kScanThreads - 1) {
+      carry_a = pa + a;
+      carry_b = pb + bt;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    list_off[n_lists] = carry_a;
+    tile_off[n_lists] = carry_b;
+  }
+}
+
+// Tile table: tile j of list L covers list rows [j * tile_m, (j+1) * tile_m).
+__global__ void regroup_tiles(int n_lists, int tile_m, const int32_t* __restrict__ counts,
+                              const int32_t* __restrict__ tile_off, int2* tiles) {
+  const int L = blockIdx.x * blockDim.x + threadIdx.x;
+  if (L >= n_lists) return;
+  const int n = (counts[L] + tile_m - 1) / tile_m;
+  const int o = tile_off[L];
+  for (int j = 0; j < n; ++j) tiles[o + j] = make_int2(L, j * tile_m);
+}
+
+}  // namespace
+
+cudaError_t launch_regroup(const Dims& dm, const Chunk& ch, const int32_t* idx, const int32_t* cu,
+                           const Regroup& rg, int* status, cudaStream_t st) {
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(rg.counts, 0, sizeof(int32_t) * ch.n_lists, st))) return e;
+  if ((e = cudaMemsetAsync(rg.cursor, 0, sizeof(int32_t) * ch.n_lists, st))) return e;
+  if (dm.batch == 0 || dm.max_seqlen == 0) {
+    return cudaMemsetAsync(rg.tile_off + ch.n_lists, 0, sizeof(int32_t), st);
+  }
+  dim3 grid((dm.max_seqlen + kThreads - 1) / kThreads, dm.batch, ch.nq);
+  regroup_pass<false><<<grid, kThreads, 0, st>>>(dm, ch, idx, cu, rg.counts, rg.cursor, nullptr,
+                                                 nullptr, status);
+  if ((e = cudaGetLastError())) return e;
+  regroup_scan<<<1, kScanThreads, 0, st>>>(ch.n_lists, ch.tile_m, rg.counts, rg.list_off,
+                                           rg.tile_off);
+  if ((e = cudaGetLastError())) return e;
+  regroup_pass<true><<<grid, kThreads, 0, st>>>(dm, ch, idx, cu, rg.counts, rg.cursor, rg.list_off,
+                                                rg.pairs, status);
+  if ((e = cudaGetLastError())) return e;
+  regroup_tiles<<<(ch.n_lists + 255) / 256, 256, 0, st>>>(ch.n_lists, ch.tile_m, rg.counts,
+                                                          rg.tile_off, rg.tiles);
+  return cudaGetLastError();
+}
+
+}  // namespace moba
