@@ -269,6 +269,9 @@ def main():
     n_pass = L.moba_num_passes(P)
     n_ev = 3 + 4 * n_pass
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    for e in evs:  # torch creates the CUDA event on first record
+        e.record(stream)
+    torch.cuda.synchronize(dev)
     ev_arr = (ctypes.c_void_p * n_ev)(*[ctypes.c_void_p(e.cuda_event) for e in evs])
     stage_ms = {"meanpool": 0.0, "gate_topk": 0.0, "regroup": 0.0, "attn_history": 0.0,
                 "attn_current": 0.0, "merge": 0.0}
