@@ -99,6 +99,26 @@ MOBA_API moba_status moba_gate_topk(const moba_params* p, const void* q, const v
                            const int32_t* cu_seqlens, int32_t* idx, void* ws, size_t ws_bytes,
                            void* stream);
 
+/* moba_gate_topk for callers that cannot allocate device memory (code
+ * running inside a runtime that owns all device memory and forbids
+ * cudaMalloc, or a latency-critical path that cannot afford cudaMalloc's
+ * device-wide synchronisation). The paper has no counterpart: this is a
+ * deployment variant of the same gate, with identical results.
+ * It needs no workspace: the block means live in a 4 MiB array compiled into
+ * the library, which every GPU that loads the library holds until the
+ * process exits. It calls no allocating routine.
+ * Limit: batch * moba_num_blocks(p) * Hkv * d * 4 bytes must not exceed
+ * 4 MiB, else MOBA_ERR_WORKSPACE is returned and nothing is launched.
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.
+ * All calls share the one array and it keeps the last call's contents
+ * (nothing in it has to start at zero); calls that overlap on the GPU --
+ * on different streams, or from different host threads -- race on it.
+ * Device-side checks of cu_seqlens are not recorded in the status word. */
+MOBA_API moba_status moba_gate_topk_noalloc(const moba_params* p, const void* q, const void* k,
+                                            const int32_t* cu_seqlens, int32_t* idx,
+                                            void* stream);
+
 /* The full forward pass: gate, regrouping of queries by the block they
  * chose, exact attention over the chosen history blocks (non-causal, eq. 6)
  * and the own block (causal, eq. 5), merged by online softmax (eq. 7-8)

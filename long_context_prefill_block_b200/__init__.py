@@ -152,6 +152,26 @@ def moba_gate_topk(q, k, cu_seqlens, block_size: int, topk: int, max_seqlen=None
     return idx
 
 
+def moba_gate_topk_noalloc(q, k, cu_seqlens, block_size: int, topk: int, max_seqlen=None,
+                           idx: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """moba_gate_topk without a workspace, for callers that cannot allocate
+    device memory: the block means use a fixed 4 MiB array inside the
+    library (see include/moba.h for the limit and the sharing rules)."""
+    _check_inputs(q, k)
+    L = lib()
+    fn = L.moba_gate_topk_noalloc
+    fn.argtypes = [ctypes.POINTER(MobaParams)] + [ctypes.c_void_p] * 5
+    fn.restype = ctypes.c_int
+    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen)
+    cu = _dev_i32(cu_seqlens, q.device)
+    if idx is None:
+        idx = torch.empty((p.total_tokens, p.num_q_heads, topk), dtype=torch.int32,
+                          device=q.device)
+    _check("moba_gate_topk_noalloc", fn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(cu), _ptr(idx),
+                                        _stream(q.device)))
+    return idx
+
+
 def moba_forward(q, k, v, cu_seqlens, block_size: int, topk: int, max_seqlen=None,
                  return_lse: bool = False, ws: Optional[torch.Tensor] = None,
                  out: Optional[torch.Tensor] = None):

@@ -1,0 +1,103 @@
+// moba_gate_topk_noalloc: the gate/top-k call for callers that cannot
+// allocate device memory.
+//
+// moba_gate_topk keeps its block means in a workspace the caller allocates.
+// Some callers cannot do that: code that runs inside a host runtime which
+// owns every byte of device memory and forbids cudaMalloc (inference
+// engines with a fixed arena, plugin interfaces of other frameworks), and
+// latency-critical paths where cudaMalloc's implicit device-wide
+// synchronisation is not acceptable. This variant takes the block means'
+// storage from a fixed array compiled into the library instead, so the
+// caller passes only inputs and outputs.
+//
+// The array below is a file-scope __device__ object: every GPU that loads
+// the library holds it until the process exits. In host code its name is
+// only a host-side stand-in, not a device address, so the device address is
+// looked up with cudaGetSymbolAddress once per device, with that device
+// current, and cached.
+#include <mutex>
+
+#include "common.cuh"
+#include "moba.h"
+
+namespace {
+
+// Largest block-mean table this entry point accepts: 4 MiB of fp32, i.e.
+// batch * ceil(max_seqlen / B) * Hkv * d <= 1,048,576 floats. The
+// million-token GQA shape (B = 4096, 8 kv heads, d = 128) needs 262,144.
+constexpr size_t kScratchBytes = size_t(4) << 20;
+
+static __device__ __align__(256) float g_gate_scratch[kScratchBytes / sizeof(float)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+float* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_gate_scratch on the current device; the first call on
+// a device performs the lookup.
+cudaError_t scratch_on_current_device(float** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_gate_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = static_cast<float*>(ptr);
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+moba_status dims_of(const moba_params* p, moba::Dims& dm) {
+  if (!p) return MOBA_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->total_tokens < 0 || p->max_seqlen < 0 || p->num_q_heads <= 0 ||
+      p->num_kv_heads <= 0 || p->num_q_heads % p->num_kv_heads != 0 || p->block_size <= 0 ||
+      p->topk <= 0)
+    return MOBA_ERR_INVALID_ARG;
+  if (p->dtype != MOBA_BF16 && p->dtype != MOBA_F32) return MOBA_ERR_UNSUPPORTED;
+  if (p->head_dim != 64 && p->head_dim != 128) return MOBA_ERR_UNSUPPORTED;
+  if (p->topk > 32) return MOBA_ERR_UNSUPPORTED;
+  if ((int64_t)p->total_tokens * p->num_q_heads * p->topk >= (int64_t(1) << 31))
+    return MOBA_ERR_UNSUPPORTED;
+  dm.batch = p->batch;
+  dm.T = p->total_tokens;
+  dm.max_seqlen = p->max_seqlen;
+  dm.Hq = p->num_q_heads;
+  dm.Hkv = p->num_kv_heads;
+  dm.d = p->head_dim;
+  dm.B = p->block_size;
+  dm.topk = p->topk;
+  dm.nb = (int)(((int64_t)p->max_seqlen + p->block_size - 1) / p->block_size);
+  dm.dtype = p->dtype == MOBA_BF16 ? moba::kBF16 : moba::kF32;
+  return MOBA_OK;
+}
+
+bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; }
+
+}  // namespace
+
+extern "C" moba_status moba_gate_topk_noalloc(const moba_params* p, const void* q, const void* k,
+                                              const int32_t* cu_seqlens, int32_t* idx,
+                                              void* stream) {
+  moba::Dims dm;
+  const moba_status s = dims_of(p, dm);
+  if (s != MOBA_OK) return s;
+  if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
+  if (!q || !k || !cu_seqlens || !idx || !aligned16(q) || !aligned16(k))
+    return MOBA_ERR_INVALID_ARG;
+  const size_t need = sizeof(float) * (size_t)dm.batch * dm.nb * dm.Hkv * dm.d;
+  if (need > kScratchBytes) return MOBA_ERR_WORKSPACE;  // beyond the built-in 4 MiB
+  float* kbar = nullptr;
+  if (scratch_on_current_device(&kbar) != cudaSuccess) return MOBA_ERR_CUDA;
+  // Nothing has to start at zero: the mean-pool writes every slot of the
+  // table that the gate reads (0 for blocks past a sequence's end).
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (moba::launch_meanpool(dm, k, cu_seqlens, kbar, nullptr, st) != cudaSuccess)
+    return MOBA_ERR_CUDA;
+  if (moba::launch_gate(dm, q, kbar, cu_seqlens, idx, nullptr, st) != cudaSuccess)
+    return MOBA_ERR_CUDA;
+  return MOBA_OK;
+}
