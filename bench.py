@@ -97,46 +97,65 @@ def profile_traffic(kernel_src: str, workload: str):
 
 # ------------------------------------------------------------ clocks
 class ClockSampler:
+    """nvidia-smi sampled every 200 ms from before the warm-up to after the
+    timed region; summarise() keeps the samples inside a wall-clock window."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
     def __init__(self, index: int):
         self.proc = None
+        self.rows = []
         self.path = tempfile.mktemp(suffix=".csv")
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
             self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}",
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={index}",
+                                          f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
+    def wait_first_sample(self, timeout=5.0):
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < timeout:
+            if os.path.getsize(self.path) > 0:
+                return
+            time.sleep(0.05)
+
     def stop(self):
         if self.proc is None:
-            return None
+            return
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
         self.f.close()
-        rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
-        os.unlink(self.path)
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
+        for line in open(self.path).read().strip().splitlines():
+            r = [x.strip() for x in line.split(",")]
             try:
-                sm.append(float(r[1]))
-                mx = max(mx, float(r[2]))
-                for nm, val in zip(names, r[5:9]):
-                    if val.strip().lower() == "active":
-                        reasons.add(nm)
+                ts = time.mktime(time.strptime(r[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + r[0].split(".")[1]) if "." in r[0] else 0.0
+                self.rows.append((ts, float(r[2]), float(r[3]), r[6:10]))
             except (ValueError, IndexError):
                 continue
-        if not sm:
+        os.unlink(self.path)
+
+    def summarise(self, t_lo: float, t_hi: float):
+        if not self.rows:
             return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        inside = [r for r in self.rows if t_lo - 0.25 <= r[0] <= t_hi + 0.25]
+        window = "timed region"
+        if not inside:
+            inside, window = self.rows, "whole run (timed region shorter than the 200 ms period)"
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({nm for r in inside for nm, val in zip(names, r[3])
+                          if val.lower() == "active"})
+        return {"sm_mhz": float(np.median([r[1] for r in inside])),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": reasons,
+                "samples": len(inside), "window": window}
 
 
 # ------------------------------------------------------------ CPU oracle leg
@@ -146,11 +165,15 @@ def time_oracle(w, q, k, v, cu, budget_s: float, seed: int = 7):
 
     qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
     total_rows = w.total_tokens * w.num_q_heads
-    n = 32
-    rows = sample_rows(total_rows, n, seed).numpy()
-    t0 = time.perf_counter()
-    oracle.forward_rows(qc, kc, vc, cu, w.block_size, w.topk, rows)
-    dt = time.perf_counter() - t0
+    n, dt = 64, 0.0
+    while True:  # grow the sample until one call takes a measurable time
+        rows = sample_rows(total_rows, n, seed).numpy()
+        t0 = time.perf_counter()
+        oracle.forward_rows(qc, kc, vc, cu, w.block_size, w.topk, rows)
+        dt = time.perf_counter() - t0
+        if dt > 0.05 * budget_s or n >= total_rows:
+            break
+        n = min(total_rows, n * 8)
     n2 = int(min(total_rows, max(n, n * budget_s / max(dt, 1e-3))))
     rows = sample_rows(total_rows, n2, seed + 1).numpy()
     t0 = time.perf_counter()
@@ -163,7 +186,7 @@ def time_oracle(w, q, k, v, cu, budget_s: float, seed: int = 7):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="scaling_8k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -244,6 +267,9 @@ def main():
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         return float(t.item())
 
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    if clocks:
+        clocks.wait_first_sample()
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize(dev)
@@ -251,17 +277,20 @@ def main():
         raise RuntimeError("device status error after warm-up")
 
     # ---- timed region: K steps, barrier + sync on both sides
-    clocks = ClockSampler(dev.index) if rank == 0 else None
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
+    t_lo = time.time()
     e0.record(stream)
     for _ in range(args.steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    t_hi = time.time()
     barrier()
-    clock_info = clocks.stop() if clocks else None
+    if clocks:
+        clocks.stop()
+    clock_info = clocks.summarise(t_lo, t_hi) if clocks else None
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
     value = useful * world / (ms * 1e-3) / 1e12
 

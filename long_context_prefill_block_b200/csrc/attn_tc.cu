@@ -11,21 +11,27 @@
 //           sequence (eq. 1, causal); writes the output.
 // The partials are combined by the merge kernel with eq. (7)-(8).
 //
-// CTA = 6 warps, one 128-row query tile:
+// Persistent CTAs (one per SM) walk a static list of 128-row query tiles.
+// Everything that a tile boundary would otherwise serialise is double
+// buffered: the query tile in shared memory (Q[2]), the logits in TMEM
+// (S[2], 128 fp32 columns each) and the output accumulator in TMEM (O[2]),
+// so the next tile's Q gather and first QK^T overlap the current tile's last
+// softmax and epilogue. Roles (8 warps):
 //   warp 0     TMA producer: K and V tiles of 128 keys (two 64-column
-//              halves each, 128-byte swizzle) into a 2-stage ring;
-//   warp 1     allocates 512 TMEM columns; lane 0 issues every tcgen05.mma:
-//              S_j = Q K_j^T into TMEM buffer j%2 (fp32, 128 columns), then
-//              O += P_{j-1} V_{j-1} with P read from TMEM (bf16 packed into
-//              the first 64 columns of the S buffer it came from);
-//   warps 2-5  softmax, one query row per thread (TMEM lane = row): load the
-//              row of S, exponentiate in base 2, store P, keep (m, l); the
-//              output accumulator O (TMEM columns 256..383) is rescaled only
-//              when a row's maximum grows by more than 2^8 (values stay
-//              below 256, exact in fp32), so PV never waits for a rescale in
-//              the common case.
-// Q rows are loaded by the softmax threads themselves (a gathered tile in
-// HIST mode) straight into the swizzled shared layout the MMA reads.
+//              halves, 128-byte swizzle) into a 2-stage ring;
+//   warp 1     allocates all 512 TMEM columns; lane 0 issues every
+//              tcgen05.mma: S = Q K^T, then O += P V for the previous KV tile
+//              with P read from TMEM (bf16, packed into the first 64 columns
+//              of the S buffer it came from);
+//   warps 2-5  softmax + epilogue, one query row per thread (TMEM lane =
+//              row): base-2 exponentials, P store, running (m, l); O is
+//              rescaled only when a row maximum grows by more than 2^8, so
+//              PV normally never waits for the softmax warps;
+//   warps 6-7  Q loaders: cp.async of the tile's (gathered, in HIST mode)
+//              query rows straight into the swizzled layout the MMA reads.
+// KV tiles are numbered globally per CTA (g); S buffer g % 2, ring stage
+// g % 2 and every barrier phase follow from g, Q/O buffers from the tile
+// count i.
 //
 // Every wait is bounded (tc::mbar_wait); on expiry the CTA records
 // kStTimeout, drains the copies and MMAs it issued, frees its TMEM and exits.
@@ -49,23 +55,27 @@ constexpr int TM = 128;   // query rows per tile
 constexpr int TN = 128;   // keys per KV tile
 constexpr int D = 128;    // head dim
 constexpr int NS = 2;     // K/V ring stages
-constexpr int kThreads = 192;
-constexpr uint32_t kHalf = 128 * 128;      // bytes of one 64-column half of a 128-row tile
-constexpr uint32_t kTile = 2 * kHalf;      // bytes of one 128 x 128 bf16 tile
-constexpr uint32_t kQOff = 0;
-constexpr uint32_t kKOff = kTile;
+constexpr int kThreads = 256;
+constexpr int kLoaderThreads = 64;
+constexpr uint32_t kHalf = 128 * 128;  // bytes of one 64-column half of a 128-row tile
+constexpr uint32_t kTile = 2 * kHalf;  // bytes of one 128 x 128 bf16 tile
+constexpr uint32_t kQOff = 0;          // Q[2]
+constexpr uint32_t kKOff = 2 * kTile;  // K[NS]
 constexpr uint32_t kVOff = kKOff + NS * kTile;
-constexpr uint32_t kSmemBytes = kVOff + NS * kTile + 1024;  // + 1024-byte alignment slack
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kOCol = 256;            // O accumulator columns [256, 384)
+constexpr uint32_t kStageRow = 144;    // bytes per staged row: 32 fp32 + 16 pad
+constexpr uint32_t kStageOff = kVOff + NS * kTile;  // epilogue staging, 32 rows per softmax warp
+constexpr uint32_t kStageBytes = 4 * 32 * kStageRow;
+constexpr uint32_t kSmemBytes = kStageOff + kStageBytes + 1024;  // + 1024-byte alignment slack
+constexpr uint32_t kTmemCols = 512;    // S[0] 0, S[1] 128, O[0] 256, O[1] 384
 constexpr uint32_t kIdescQK = idesc_bf16(TM, TN, false, false);  // Q, K both K-major
 constexpr uint32_t kIdescPV = idesc_bf16(TM, D, false, true);    // V is MN-major (d contiguous)
 constexpr float kRescaleLog2 = 8.f;
 
 struct Shared {
-  uint64_t q_full;
+  uint64_t q_full[2], q_empty[2];
   uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
   uint64_t s_full[2], s_free[2], p_full[2];
+  uint64_t o_full[2], o_free[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -76,6 +86,7 @@ struct Args {
   Chunk ch;
   const __nv_bfloat16* q;
   const int32_t* cu;
+  int n_tiles;  // CUR / DENSE: size of the static tile space
   // HIST
   const int32_t* list_off;
   const int32_t* pairs;
@@ -91,6 +102,119 @@ struct Args {
   int* status;
 };
 
+struct Tile {
+  bool skip;
+  int b, g, h, kv0, n_kv, p0, list, row0, count;
+  int64_t start;
+};
+
+// Tile t of the static tile space. CUR / DENSE tiles are ordered longest
+// first so the persistent CTAs end together.
+template <int MODE>
+__device__ __forceinline__ Tile get_tile(const Args& a, int t) {
+  const Dims& dm = a.dm;
+  Tile T{};
+  T.skip = false;
+  if (MODE == HIST) {
+    const int2 tl = a.tiles[t];
+    T.list = tl.x;
+    T.row0 = tl.y;
+    const int e = T.list % dm.nb;
+    T.g = a.ch.g0 + (T.list / dm.nb) % a.ch.ng;
+    T.b = T.list / (dm.nb * a.ch.ng);
+    T.count = a.list_off[T.list + 1] - a.list_off[T.list];
+    T.kv0 = e * dm.B;
+    T.n_kv = dm.B / TN;
+    T.start = a.cu[T.b];
+    return T;
+  }
+  int qt;
+  if (MODE == CUR) {
+    const int R = dm.B / TM;                      // query tiles per block
+    const int per = dm.nb * dm.batch * a.ch.nq;   // tiles with the same r
+    const int r = R - 1 - t / per;
+    int rem = t % per;
+    const int c = rem / (dm.batch * a.ch.nq);
+    rem %= dm.batch * a.ch.nq;
+    T.b = rem / a.ch.nq;
+    T.h = a.ch.h0 + rem % a.ch.nq;
+    T.p0 = c * dm.B + r * TM;
+    T.kv0 = c * dm.B;
+    T.n_kv = r + 1;
+    qt = 0;
+  } else {
+    const int nqt = (dm.max_seqlen + TM - 1) / TM;
+    const int per = dm.batch * dm.Hq;
+    qt = nqt - 1 - t / per;
+    const int rem = t % per;
+    T.b = rem / dm.Hq;
+    T.h = rem % dm.Hq;
+    T.p0 = qt * TM;
+    T.kv0 = 0;
+    T.n_kv = qt + 1;
+  }
+  T.g = T.h / (dm.Hq / dm.Hkv);
+  T.start = a.cu[T.b];
+  const int len = a.cu[T.b + 1] - a.cu[T.b];
+  T.count = len;  // sequence length, for the row checks below
+  T.skip = len < 0 || len > dm.max_seqlen || T.p0 >= len;
+  return T;
+}
+
+// Identity of query row r of a tile: the q row it reads (t * Hq + h, or -1)
+// and, for outputs, the token t, head h, position p and partial row prow.
+struct Row {
+  bool has_q, valid;
+  int64_t t, prow;
+  int h, p;
+};
+
+template <int MODE>
+__device__ __forceinline__ Row get_row(const Args& a, const Tile& T, int r) {
+  const Dims& dm = a.dm;
+  Row R{};
+  if (MODE == HIST) {
+    R.has_q = R.valid = T.row0 + r < T.count;
+    if (R.valid) {
+      R.prow = a.pairs[a.list_off[T.list] + T.row0 + r];
+      const int64_t th = R.prow / dm.topk;
+      R.t = th / a.ch.nq;
+      R.h = a.ch.h0 + (int)(th % a.ch.nq);
+    }
+    return R;
+  }
+  R.h = T.h;
+  R.p = T.p0 + r;
+  R.has_q = R.valid = R.p < T.count;
+  R.t = T.start + R.p;
+  if (MODE == CUR && R.valid) {
+    const int c = R.p / dm.B;
+    const int32_t* row = a.idx + (R.t * dm.Hq + R.h) * (int64_t)dm.topk;
+    int slot = -1;
+    for (int i = 0; i < dm.topk; ++i)
+      if (row[i] == c && slot < 0) slot = i;
+    R.prow = (R.t * a.ch.nq + (R.h - a.ch.h0)) * (int64_t)dm.topk + (slot < 0 ? 0 : slot);
+    R.valid = slot >= 0;
+  }
+  return R;
+}
+
+// Query row r of a tile for the loader: the q row it reads, or none.
+template <int MODE>
+__device__ __forceinline__ bool q_row_of(const Args& a, const Tile& T, int r, int64_t& qrow) {
+  if (MODE == HIST) {
+    if (T.row0 + r >= T.count) return false;
+    const int64_t prow = a.pairs[a.list_off[T.list] + T.row0 + r];
+    const int64_t th = prow / a.dm.topk;
+    qrow = (th / a.ch.nq) * a.dm.Hq + a.ch.h0 + (int)(th % a.ch.nq);
+    return true;
+  }
+  const int p = T.p0 + r;
+  if (p >= T.count) return false;
+  qrow = (T.start + p) * a.dm.Hq + T.h;
+  return true;
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -99,55 +223,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
   __shared__ Shared sh;
   const Dims& dm = a.dm;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // ---- which tile ----------------------------------------------------------
-  int b, g, n_kv, kv0;   // sequence, kv head, KV tiles, first key (sequence-relative)
-  int p0 = 0;            // first query position (CUR / DENSE)
-  int h_fixed = 0;       // q head (CUR / DENSE)
-  int list = 0, row0 = 0, count = 0;
   if (a.status && *reinterpret_cast<volatile int*>(a.status) == kStTimeout) return;
-  if (MODE == HIST) {
-    if ((int)blockIdx.x >= *a.tile_count) return;
-    const int2 tl = a.tiles[blockIdx.x];
-    list = tl.x;
-    row0 = tl.y;
-    const int e = list % dm.nb;
-    g = a.ch.g0 + (list / dm.nb) % a.ch.ng;
-    b = list / (dm.nb * a.ch.ng);
-    count = a.list_off[list + 1] - a.list_off[list];
-    kv0 = e * dm.B;
-    n_kv = dm.B / TN;
-  } else {
-    b = blockIdx.y;
-    const int len = a.cu[b + 1] - a.cu[b];
-    if (len < 0 || len > dm.max_seqlen) return;
-    // longest tiles first (they end last)
-    const int qt = gridDim.x - 1 - blockIdx.x;
-    p0 = qt * TM;
-    if (p0 >= len) return;
-    h_fixed = (MODE == CUR ? a.ch.h0 : 0) + blockIdx.z;
-    g = h_fixed / (dm.Hq / dm.Hkv);
-    const int c = p0 / dm.B;
-    kv0 = MODE == CUR ? c * dm.B : 0;
-    n_kv = (p0 - kv0) / TN + 1;
-  }
-  const int64_t start = a.cu[b];
+  const int n_tiles = MODE == HIST ? *a.tile_count : a.n_tiles;
+  if ((int)blockIdx.x >= n_tiles) return;
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sQ = sbase + kQOff, sK = sbase + kKOff, sV = sbase + kVOff;
 
   if (threadIdx.x == 0) {
-    mbar_init(&sh.q_full, 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.q_full[i], kLoaderThreads);
+      mbar_init(&sh.q_empty[i], 1);
+      mbar_init(&sh.s_full[i], 1);
+      mbar_init(&sh.s_free[i], 1);
+      mbar_init(&sh.p_full[i], 128);
+      mbar_init(&sh.o_full[i], 1);
+      mbar_init(&sh.o_free[i], 128);
+    }
     for (int i = 0; i < NS; ++i) {
       mbar_init(&sh.k_full[i], 1);
       mbar_init(&sh.k_empty[i], 1);
       mbar_init(&sh.v_full[i], 1);
       mbar_init(&sh.v_empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sh.s_full[i], 1);
-      mbar_init(&sh.s_free[i], 1);
-      mbar_init(&sh.p_full[i], 128);
     }
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
@@ -162,243 +259,319 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
   fence_after_sync();
   const uint32_t tmem = sh.tmem_base;
   volatile int* abort = &sh.abort;
+  int* status = a.status;
 
   if (warp == 0) {
-    // ================= TMA producer =================
+    // ================= TMA producer: K and V tiles =================
     if (lane == 0) {
-      int issued_k = 0, issued_v = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int st = j % NS, u = j / NS;
-        const int z = (int)(start + kv0 + j * TN);
-        if (u > 0 && !mbar_wait(&sh.k_empty[st], (u - 1) & 1, abort, a.status)) break;
-        mbar_expect_tx(&sh.k_full[st], kTile);
-        tma_load_3d(sK + st * kTile, &tmk, &sh.k_full[st], 0, g, z);
-        tma_load_3d(sK + st * kTile + kHalf, &tmk, &sh.k_full[st], 64, g, z);
-        issued_k = j + 1;
-        if (u > 0 && !mbar_wait(&sh.v_empty[st], (u - 1) & 1, abort, a.status)) break;
-        mbar_expect_tx(&sh.v_full[st], kTile);
-        tma_load_3d(sV + st * kTile, &tmv, &sh.v_full[st], 0, g, z);
-        tma_load_3d(sV + st * kTile + kHalf, &tmv, &sh.v_full[st], 64, g, z);
-        issued_v = j + 1;
+      uint32_t g = 0, nk = 0, nv = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+        const Tile T = get_tile<MODE>(a, t);
+        if (T.skip) continue;
+        for (int j = 0; j < T.n_kv; ++j, ++g) {
+          const uint32_t st = g % NS, u = g / NS;
+          const int z = (int)(T.start + T.kv0 + j * TN);
+          if (u > 0 && !(ok = mbar_wait(&sh.k_empty[st], (u - 1) & 1, abort, status))) break;
+          mbar_expect_tx(&sh.k_full[st], kTile);
+          tma_load_3d(sK + st * kTile, &tmk, &sh.k_full[st], 0, T.g, z);
+          tma_load_3d(sK + st * kTile + kHalf, &tmk, &sh.k_full[st], 64, T.g, z);
+          nk = g + 1;
+          if (u > 0 && !(ok = mbar_wait(&sh.v_empty[st], (u - 1) & 1, abort, status))) break;
+          mbar_expect_tx(&sh.v_full[st], kTile);
+          tma_load_3d(sV + st * kTile, &tmv, &sh.v_full[st], 0, T.g, z);
+          tma_load_3d(sV + st * kTile + kHalf, &tmv, &sh.v_full[st], 64, T.g, z);
+          nv = g + 1;
+        }
       }
-      if (*abort) {
+      if (!ok || *abort) {
         // let the copies already issued land before the CTA exits
-        for (int j = (issued_k > NS ? issued_k - NS : 0); j < issued_k; ++j)
-          mbar_drain(&sh.k_full[j % NS], (j / NS) & 1);
-        for (int j = (issued_v > NS ? issued_v - NS : 0); j < issued_v; ++j)
-          mbar_drain(&sh.v_full[j % NS], (j / NS) & 1);
+        for (uint32_t x = nk > NS ? nk - NS : 0; x < nk; ++x)
+          mbar_drain(&sh.k_full[x % NS], (x / NS) & 1);
+        for (uint32_t x = nv > NS ? nv - NS : 0; x < nv; ++x)
+          mbar_drain(&sh.v_full[x % NS], (x / NS) & 1);
       }
     }
   } else if (warp == 1) {
     // ================= MMA issuer =================
     if (lane == 0) {
-      const uint32_t tS[2] = {tmem, tmem + 128};
-      const uint32_t tO = tmem + kOCol;
-      bool ok = mbar_wait(&sh.q_full, 0, abort, a.status);
-      auto issue_pv = [&](int jj) -> bool {
-        const int st = jj % NS, bb = jj & 1;
-        if (!mbar_wait(&sh.p_full[bb], (jj >> 1) & 1, abort, a.status)) return false;
-        if (!mbar_wait(&sh.v_full[st], (jj / NS) & 1, abort, a.status)) return false;
+      const uint32_t tS0 = tmem, tO0 = tmem + 256;
+      uint32_t g = 0, i = 0;
+      bool ok = true, pend = false, plast = false;
+      uint32_t pg = 0, pi = 0;
+      int pj = 0;
+      auto issue_pv = [&](uint32_t gg, uint32_t ii, int jj, bool last) -> bool {
+        const uint32_t ob = ii & 1, bb = gg & 1, st = gg % NS;
+        if (jj == 0 && ii >= 2 && !mbar_wait(&sh.o_free[ob], ((ii >> 1) - 1) & 1, abort, status))
+          return false;
+        if (!mbar_wait(&sh.p_full[bb], (gg >> 1) & 1, abort, status)) return false;
+        if (!mbar_wait(&sh.v_full[st], (gg / NS) & 1, abort, status)) return false;
         fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < TN / 16; ++kk) {
           const uint64_t bd = desc_sw128(sV + st * kTile + kk * 16 * 128, kHalf, 1024);
-          mma_ts(tO, tS[bb] + kk * 8, bd, kIdescPV, (jj > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tO0 + ob * 128, tS0 + bb * 128 + kk * 8, bd, kIdescPV,
+                 (jj > 0 || kk > 0) ? 1u : 0u);
         }
         commit(&sh.v_empty[st]);
         commit(&sh.s_free[bb]);
+        if (last) commit(&sh.o_full[ob]);
         return true;
       };
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int st = j % NS, bb = j & 1;
-        if (!mbar_wait(&sh.k_full[st], (j / NS) & 1, abort, a.status)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait(&sh.s_free[bb], ((j - 2) >> 1) & 1, abort, a.status)) {
-          ok = false;
-          break;
-        }
-        fence_after_sync();
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+        const Tile T = get_tile<MODE>(a, t);
+        if (T.skip) continue;
+        const uint32_t qb = i & 1;
+        if (!(ok = mbar_wait(&sh.q_full[qb], (i >> 1) & 1, abort, status))) break;
+        for (int j = 0; j < T.n_kv; ++j, ++g) {
+          const uint32_t st = g % NS, bb = g & 1;
+          if (!(ok = mbar_wait(&sh.k_full[st], (g / NS) & 1, abort, status))) break;
+          if (g >= 2 && !(ok = mbar_wait(&sh.s_free[bb], ((g - 2) >> 1) & 1, abort, status)))
+            break;
+          fence_after_sync();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          const uint64_t ad = desc_sw128(sQ + off, 16, 1024);
-          const uint64_t bd = desc_sw128(sK + st * kTile + off, 16, 1024);
-          mma_ss(tS[bb], ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+            const uint64_t ad = desc_sw128(sQ + qb * kTile + off, 16, 1024);
+            const uint64_t bd = desc_sw128(sK + st * kTile + off, 16, 1024);
+            mma_ss(tS0 + bb * 128, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
+          }
+          commit(&sh.s_full[bb]);
+          commit(&sh.k_empty[st]);
+          if (j == T.n_kv - 1) commit(&sh.q_empty[qb]);
+          if (pend && !(ok = issue_pv(pg, pi, pj, plast))) break;
+          pend = true;
+          pg = g;
+          pi = i;
+          pj = j;
+          plast = j == T.n_kv - 1;
         }
-        commit(&sh.s_full[bb]);
-        commit(&sh.k_empty[st]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        ++i;
       }
-      if (ok) ok = issue_pv(n_kv - 1);
+      if (ok && pend) ok = issue_pv(pg, pi, pj, plast);
       if (!ok) {
         // wait until every MMA issued so far has finished
         commit(&sh.drain);
         mbar_drain(&sh.drain, 0);
       }
     }
-  } else {
-    // ================= softmax warps 2..5 =================
+  } else if (warp < 6) {
+    // ================= softmax + epilogue, warps 2..5 =================
     const int quarter = warp & 3;          // TMEM lanes this warp may access
     const int r = quarter * 32 + lane;     // query row of this thread
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    // row identity
-    bool valid = false;
-    int64_t t = 0, prow = 0;
-    int h = h_fixed, p = 0;
-    if (MODE == HIST) {
-      valid = row0 + r < count;
-      if (valid) {
-        prow = a.pairs[a.list_off[list] + row0 + r];
-        const int64_t th = prow / dm.topk;
-        t = th / a.ch.nq;
-        h = a.ch.h0 + (int)(th % a.ch.nq);
-      }
-    } else {
-      const int len = a.cu[b + 1] - a.cu[b];
-      p = p0 + r;
-      valid = p < len;
-      t = start + p;
-      if (MODE == CUR && valid) {
-        const int c = p / dm.B;
-        const int32_t* row = a.idx + (t * dm.Hq + h) * (int64_t)dm.topk;
-        int slot = -1;
-        for (int i = 0; i < dm.topk; ++i)
-          if (row[i] == c && slot < 0) slot = i;
-        prow = (t * a.ch.nq + (h - a.ch.h0)) * (int64_t)dm.topk + (slot < 0 ? 0 : slot);
-        valid = slot >= 0;
-      }
-    }
-    const bool has_q = MODE == HIST ? (row0 + r < count) : (p < a.cu[b + 1] - a.cu[b]);
-    // ---- Q row -> swizzled shared tile (two 64-column halves)
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(a.q + (t * dm.Hq + h) * (int64_t)D);
-#pragma unroll
-      for (int c16 = 0; c16 < 16; ++c16) {
-        const uint4 x = has_q ? __ldg(src + c16) : make_uint4(0, 0, 0, 0);
-        const uint32_t half = c16 >> 3, cc = c16 & 7;
-        const uint32_t addr = sQ + half * kHalf + r * 128 + ((cc ^ (r & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x.x),
-                     "r"(x.y), "r"(x.z), "r"(x.w)
-                     : "memory");
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&sh.q_full);
-    }
     const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;  // softmax scale, base 2
-    float m_i = -INFINITY, l_i = 0.f;
+    uint32_t g = 0, i = 0;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int bb = j & 1;
-      ok = mbar_wait(&sh.s_full[bb], (j >> 1) & 1, abort, a.status);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      fence_after_sync();
-      const uint32_t tS = tmem + bb * 128 + lane_addr;
-      float s[TN];
-#pragma unroll
-      for (int c = 0; c < TN / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(tS + c * 32, rr);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(rr[i]) * sl2;
-      }
-      // causal mask on the diagonal tile (CUR / DENSE): key > query
-      if (MODE != HIST && j == n_kv - 1) {
-        const int lim = p - (kv0 + j * TN);  // last visible column
-#pragma unroll
-        for (int i = 0; i < TN; ++i)
-          if (i > lim) s[i] = -INFINITY;
-      }
-      float mt = s[0];
-#pragma unroll
-      for (int i = 1; i < TN; ++i) mt = fmaxf(mt, s[i]);
-      const bool need = mt > m_i + kRescaleLog2;
-      const float m_new = need ? mt : m_i;
-      if (__any_sync(0xffffffffu, need) && j > 0) {
-        // O holds PV of tiles < j: wait until PV_{j-1} has landed, then rescale
-        ok = mbar_wait(&sh.s_free[(j - 1) & 1], ((j - 1) >> 1) & 1, abort, a.status);
+    for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+      const Tile T = get_tile<MODE>(a, t);
+      if (T.skip) continue;
+      const Row R = get_row<MODE>(a, T, r);
+      const uint32_t ob = i & 1;
+      const uint32_t tO = tmem + 256 + ob * 128 + lane_addr;
+      float m_i = -INFINITY, l_i = 0.f;
+      for (int j = 0; j < T.n_kv; ++j, ++g) {
+        const uint32_t bb = g & 1;
+        ok = mbar_wait(&sh.s_full[bb], (g >> 1) & 1, abort, status);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         fence_after_sync();
-        const float alpha = need ? ex2(m_i - m_new) : 1.f;
-        const uint32_t tO = tmem + kOCol + lane_addr;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t rr[32];
-          tmem_ld32(tO + c * 32, rr);
+        const uint32_t tS = tmem + bb * 128 + lane_addr;
+        float s[TN];
+        {
+          // issue all four loads, then one wait
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          tmem_ld32(tS, r0);
+          tmem_ld32(tS + 32, r1);
+          tmem_ld32(tS + 64, r2);
+          tmem_ld32(tS + 96, r3);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-          tmem_st32(tO + c * 32, rr);
+          for (int x = 0; x < 32; ++x) {
+            s[x] = __uint_as_float(r0[x]);
+            s[32 + x] = __uint_as_float(r1[x]);
+            s[64 + x] = __uint_as_float(r2[x]);
+            s[96 + x] = __uint_as_float(r3[x]);
+          }
+        }
+        // causal mask on the diagonal tile (CUR / DENSE): key > query
+        if (MODE != HIST && j == T.n_kv - 1) {
+          const int lim = R.p - (T.kv0 + j * TN);  // last visible column
+#pragma unroll
+          for (int x = 0; x < TN; ++x)
+            if (x > lim) s[x] = -INFINITY;
+        }
+        // row maximum as a tree of 8 independent chains
+        float mv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mv[u] = s[u];
+#pragma unroll
+        for (int x = 8; x < TN; x += 8)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mv[u] = fmaxf(mv[u], s[x + u]);
+        const float mx = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
+                               fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
+        const float mt = mx * sl2;
+        const bool need = mt > m_i + kRescaleLog2;
+        const float m_new = need ? mt : m_i;
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // O holds PV of this tile's earlier KV tiles: wait for the last, rescale
+          ok = mbar_wait(&sh.s_free[(g - 1) & 1], ((g - 1) >> 1) & 1, abort, status);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          fence_after_sync();
+          const float alpha = need ? ex2(m_i - m_new) : 1.f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t rr[32];
+            tmem_ld32(tO + c * 32, rr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) rr[x] = __float_as_uint(__uint_as_float(rr[x]) * alpha);
+            tmem_st32(tO + c * 32, rr);
+          }
+          tmem_wait_st();
+        }
+        if (need) {
+          l_i *= ex2(m_i - m_new);
+          m_i = m_new;
+        }
+        // P = exp2(s * scale - m) in bf16, two per column, into the S buffer;
+        // the row sum is kept in 8 independent partial sums
+        float ps[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) ps[u] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            const float e0 = ex2(fmaf(s[c * 64 + 2 * x], sl2, -m_i));
+            const float e1 = ex2(fmaf(s[c * 64 + 2 * x + 1], sl2, -m_i));
+            ps[(2 * x) & 7] += e0;
+            ps[(2 * x + 1) & 7] += e1;
+            pk[x] = pack_bf16x2(e0, e1);
+          }
+          tmem_st32(tS + c * 32, pk);
         }
         tmem_wait_st();
+        const float rowsum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        l_i += rowsum;
+        fence_before_sync();
+        mbar_arrive(&sh.p_full[bb]);
       }
-      if (need) {
-        l_i *= ex2(m_i - m_new);
-        m_i = m_new;
-      }
-      // P = exp2(s - m) in bf16, packed two per column into the S buffer
-      float rowsum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float e0 = ex2(s[c * 64 + 2 * i] - m_i);
-          const float e1 = ex2(s[c * 64 + 2 * i + 1] - m_i);
-          rowsum += e0 + e1;
-          pk[i] = pack_bf16x2(e0, e1);
-        }
-        tmem_st32(tS + c * 32, pk);
-      }
-      tmem_wait_st();
-      l_i += rowsum;
-      fence_before_sync();
-      mbar_arrive(&sh.p_full[bb]);
-    }
-    // ---- epilogue: wait for the last PV, normalise, write
-    if (ok) {
-      const int jl = n_kv - 1;
-      ok = mbar_wait(&sh.s_free[jl & 1], (jl >> 1) & 1, abort, a.status);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
+      if (!ok) break;
+      // ---- epilogue: wait for the tile's last PV, normalise, write
+      ok = mbar_wait(&sh.o_full[ob], (i >> 1) & 1, abort, status);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       fence_after_sync();
       const float inv_l = 1.f / l_i;
       const float lse = (m_i + log2f(l_i)) * 0.6931471805599453f;
-      const uint32_t tO = tmem + kOCol + lane_addr;
-#pragma unroll
+      // Rows go out through a per-warp staging area so that every global
+      // store instruction writes whole 128-byte segments of 4 or 8 rows.
+      const uint32_t stage = sbase + kStageOff + (warp - 2) * 32 * kStageRow;
+      const int64_t orow = R.valid ? (MODE == DENSE ? R.t * dm.Hq + R.h : R.prow) : -1;
+#pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t rr[32];
         tmem_ld32(tO + c * 32, rr);
         tmem_wait_ld();
-        if (valid) {
-          if (MODE == DENSE) {
-            uint32_t pk[16];
+        if (MODE == DENSE) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = pack_bf16x2(__uint_as_float(rr[2 * i]) * inv_l,
-                                  __uint_as_float(rr[2 * i + 1]) * inv_l);
-            uint4* dst = reinterpret_cast<uint4*>(a.out + (t * dm.Hq + h) * (int64_t)D + c * 32);
+          for (int x = 0; x < 4; ++x) {
+            const uint32_t w0 = pack_bf16x2(__uint_as_float(rr[8 * x]) * inv_l,
+                                            __uint_as_float(rr[8 * x + 1]) * inv_l);
+            const uint32_t w1 = pack_bf16x2(__uint_as_float(rr[8 * x + 2]) * inv_l,
+                                            __uint_as_float(rr[8 * x + 3]) * inv_l);
+            const uint32_t w2 = pack_bf16x2(__uint_as_float(rr[8 * x + 4]) * inv_l,
+                                            __uint_as_float(rr[8 * x + 5]) * inv_l);
+            const uint32_t w3 = pack_bf16x2(__uint_as_float(rr[8 * x + 6]) * inv_l,
+                                            __uint_as_float(rr[8 * x + 7]) * inv_l);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             stage + lane * 80 + x * 16),
+                         "r"(w0), "r"(w1), "r"(w2), "r"(w3)
+                         : "memory");
+          }
+          __syncwarp();
+          // 64 bytes per row chunk: 4 lanes per row, 8 rows per instruction
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-          } else {
-            float4* dst = reinterpret_cast<float4*>(a.part_o + prow * D + c * 32);
+          for (int it = 0; it < 4; ++it) {
+            const int row = it * 8 + (lane >> 2), seg = lane & 3;
+            const int64_t o = __shfl_sync(0xffffffffu, orow, row);
+            uint4 val;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                         : "r"(stage + row * 80 + seg * 16)
+                         : "memory");
+            if (o >= 0)
+              *reinterpret_cast<uint4*>(a.out + o * D + c * 32 + seg * 8) = val;
+          }
+        } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(rr[4 * i]) * inv_l,
-                                   __uint_as_float(rr[4 * i + 1]) * inv_l,
-                                   __uint_as_float(rr[4 * i + 2]) * inv_l,
-                                   __uint_as_float(rr[4 * i + 3]) * inv_l);
+          for (int x = 0; x < 8; ++x)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             stage + lane * kStageRow + x * 16),
+                         "r"(__float_as_uint(__uint_as_float(rr[4 * x]) * inv_l)),
+                         "r"(__float_as_uint(__uint_as_float(rr[4 * x + 1]) * inv_l)),
+                         "r"(__float_as_uint(__uint_as_float(rr[4 * x + 2]) * inv_l)),
+                         "r"(__float_as_uint(__uint_as_float(rr[4 * x + 3]) * inv_l))
+                         : "memory");
+          __syncwarp();
+          // 128 bytes per row chunk: 8 lanes per row, 4 rows per instruction
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int row = it * 4 + (lane >> 3), seg = lane & 7;
+            const int64_t o = __shfl_sync(0xffffffffu, orow, row);
+            uint4 val;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                         : "r"(stage + row * kStageRow + seg * 16)
+                         : "memory");
+            if (o >= 0)
+              *reinterpret_cast<uint4*>(a.part_o + o * D + c * 32 + seg * 4) = val;
           }
         }
+        __syncwarp();
       }
-      if (valid) {
+      if (R.valid) {
         if (MODE == DENSE) {
-          if (a.lse_out) a.lse_out[t * dm.Hq + h] = lse;
+          if (a.lse_out) a.lse_out[R.t * dm.Hq + R.h] = lse;
         } else {
-          a.part_lse[prow] = lse;
+          a.part_lse[R.prow] = lse;
         }
       }
+      fence_before_sync();
+      mbar_arrive(&sh.o_free[ob]);
+      ++i;
+    }
+  } else {
+    // ================= Q loaders, warps 6..7 =================
+    const int tl = threadIdx.x - (kThreads - kLoaderThreads);
+    uint32_t i = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+      const Tile T = get_tile<MODE>(a, t);
+      if (T.skip) continue;
+      const uint32_t qb = i & 1;
+      if (i >= 2) {
+        ok = mbar_wait(&sh.q_empty[qb], ((i >> 1) - 1) & 1, abort, status);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      }
+#pragma unroll
+      for (int half_rows = 0; half_rows < TM / kLoaderThreads; ++half_rows) {
+        const int rr = tl + half_rows * kLoaderThreads;
+        int64_t qrow = 0;
+        const bool has = q_row_of<MODE>(a, T, rr, qrow);
+        const __nv_bfloat16* src = a.q + (has ? qrow : 0) * (int64_t)D;
+#pragma unroll
+        for (int c16 = 0; c16 < 16; ++c16) {
+          const uint32_t dst = sQ + qb * kTile + (c16 >> 3) * kHalf + rr * 128 +
+                               ((((uint32_t)c16 & 7u) ^ ((uint32_t)rr & 7u)) << 4);
+          cp_async16(dst, src + c16 * 8, has ? 16u : 0u);
+        }
+      }
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      mbar_arrive(&sh.q_full[qb]);
+      ++i;
     }
   }
 
@@ -439,8 +612,17 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int T, int H) {
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n > 0 ? n : 148;
+}
+
 template <int MODE>
-cudaError_t launch(dim3 grid, const Args& args, const void* k, const void* v, cudaStream_t st) {
+cudaError_t launch(int64_t tiles, const Args& args, const void* k, const void* v,
+                   cudaStream_t st) {
+  if (tiles <= 0) return cudaSuccess;
   CUtensorMap mk, mv;
   cudaError_t e;
   if ((e = make_map(&mk, k, args.dm.T, args.dm.Hkv))) return e;
@@ -448,7 +630,8 @@ cudaError_t launch(dim3 grid, const Args& args, const void* k, const void* v, cu
   if ((e = cudaFuncSetAttribute(attn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 kSmemBytes)))
     return e;
-  attn_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(mk, mv, args);
+  const int64_t grid = tiles < sm_count() ? tiles : sm_count();
+  attn_tc_kernel<MODE><<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mk, mv, args);
   return cudaGetLastError();
 }
 
@@ -467,7 +650,6 @@ Args base_args(const Dims& dm, const Chunk& ch, const void* q, const int32_t* cu
 cudaError_t launch_history_tc(const Dims& dm, const Chunk& ch, const void* q, const void* k,
                               const void* v, const int32_t* cu, const Regroup& rg,
                               const Partials& pt, int* status, cudaStream_t st) {
-  if (rg.max_tiles == 0) return cudaSuccess;
   Args a = base_args(dm, ch, q, cu, status);
   a.list_off = rg.list_off;
   a.pairs = rg.pairs;
@@ -475,7 +657,7 @@ cudaError_t launch_history_tc(const Dims& dm, const Chunk& ch, const void* q, co
   a.tile_count = rg.tile_off + ch.n_lists;
   a.part_o = pt.o;
   a.part_lse = pt.lse;
-  return launch<HIST>(dim3((unsigned)rg.max_tiles), a, k, v, st);
+  return launch<HIST>(rg.max_tiles, a, k, v, st);
 }
 
 cudaError_t launch_current_tc(const Dims& dm, const Chunk& ch, const void* q, const void* k,
@@ -486,7 +668,9 @@ cudaError_t launch_current_tc(const Dims& dm, const Chunk& ch, const void* q, co
   a.idx = idx;
   a.part_o = pt.o;
   a.part_lse = pt.lse;
-  return launch<CUR>(dim3((dm.max_seqlen + TM - 1) / TM, dm.batch, ch.nq), a, k, v, st);
+  const int64_t tiles = (int64_t)(dm.B / TM) * dm.nb * dm.batch * ch.nq;
+  a.n_tiles = (int)tiles;
+  return launch<CUR>(tiles, a, k, v, st);
 }
 
 cudaError_t launch_dense_tc(const Dims& dm, const void* q, const void* k, const void* v,
@@ -497,7 +681,9 @@ cudaError_t launch_dense_tc(const Dims& dm, const void* q, const void* k, const 
   Args a = base_args(dm, ch, q, cu, status);
   a.out = static_cast<__nv_bfloat16*>(out);
   a.lse_out = lse;
-  return launch<DENSE>(dim3((dm.max_seqlen + TM - 1) / TM, dm.batch, dm.Hq), a, k, v, st);
+  const int64_t tiles = (int64_t)((dm.max_seqlen + TM - 1) / TM) * dm.batch * dm.Hq;
+  a.n_tiles = (int)tiles;
+  return launch<DENSE>(tiles, a, k, v, st);
 }
 
 }  // namespace moba

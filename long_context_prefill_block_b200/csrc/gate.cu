@@ -8,10 +8,12 @@
 //
 // Scores are fp32 FMA (q widened from bf16, kbar fp32): the near-tie band of
 // the parity check is 1e-4 relative and bf16/tf32 products would flip far
-// more ranks than that. One CTA scores 32 queries of one (sequence, head);
-// 4 threads per query each scan a quarter of every 32-block chunk of kbar
-// held in shared memory and keep a sorted register list of their best
-// KM >= k-1 blocks; the four lists are merged by warp shuffles.
+// more ranks than that. One CTA scores 64 consecutive queries of one
+// (sequence, head) against the earlier blocks in chunks of 32: a register-
+// tiled fp32 GEMM (each thread 4 queries x 2 blocks, operands in shared
+// memory) writes the chunk's scores to shared memory, then 4 threads per
+// query scan them into sorted register lists of their best KM >= k-1
+// blocks; at the end the four lists are merged by warp shuffles.
 #include <climits>
 #include <cmath>
 
@@ -20,8 +22,8 @@
 namespace moba {
 namespace {
 
-constexpr int kQ = 32;        // queries per CTA
-constexpr int kThreads = 128; // 4 threads per query
+constexpr int kQ = 64;        // queries per CTA
+constexpr int kThreads = 256; // 4 threads per query in the selection phase
 constexpr int kCh = 32;       // kbar rows per shared-memory chunk
 
 __device__ __forceinline__ bool better(float s, int i, float t, int j) {
@@ -48,8 +50,10 @@ __global__ void __launch_bounds__(kThreads) gate_kernel(Dims dm, const T* __rest
                                                         const float* __restrict__ kbar,
                                                         const int32_t* __restrict__ cu,
                                                         int32_t* __restrict__ idx, int* status) {
-  __shared__ __align__(16) float qs[kQ][D + 4];
-  __shared__ __align__(16) float kb[kCh][D + 4];
+  extern __shared__ __align__(16) float gsm[];
+  float(*qs)[D + 4] = reinterpret_cast<float(*)[D + 4]>(gsm);                     // [kQ]
+  float(*kb)[D + 4] = reinterpret_cast<float(*)[D + 4]>(gsm + kQ * (D + 4));      // [kCh]
+  float(*sc)[kCh + 1] = reinterpret_cast<float(*)[kCh + 1]>(gsm + (kQ + kCh) * (D + 4));
 
   const int b = blockIdx.y, h = blockIdx.z;
   const int g = h / (dm.Hq / dm.Hkv);
@@ -73,7 +77,10 @@ __global__ void __launch_bounds__(kThreads) gate_kernel(Dims dm, const T* __rest
     for (int u = 0; u < VEC; ++u) qs[r][l * VEC + u] = x[u];
   }
 
+  // selection mapping: query qi, quarter `part` of every chunk
   const int qi = threadIdx.x >> 2, part = threadIdx.x & 3;
+  // GEMM mapping: queries ty + 16 i (i < 4), blocks tx + 16 j (j < 2)
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
   const int p = p0 + qi;
   const bool valid = p < len;
   const int c = valid ? p / dm.B : 0;
@@ -90,33 +97,45 @@ __global__ void __launch_bounds__(kThreads) gate_kernel(Dims dm, const T* __rest
   for (int base = 0; base < cmax; base += kCh) {
     __syncthreads();
     const int nblk = min(kCh, cmax - base);
-    for (int e = threadIdx.x; e < nblk * (D / 4); e += kThreads) {
+    for (int e = threadIdx.x; e < kCh * (D / 4); e += kThreads) {
       const int r = e / (D / 4), l = e % (D / 4);
-      *reinterpret_cast<float4*>(&kb[r][l * 4]) = __ldg(reinterpret_cast<const float4*>(
-          kbar + (((int64_t)b * dm.nb + base + r) * dm.Hkv + g) * D + l * 4));
+      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < nblk)
+        w = __ldg(reinterpret_cast<const float4*>(
+            kbar + (((int64_t)b * dm.nb + base + r) * dm.Hkv + g) * D + l * 4));
+      *reinterpret_cast<float4*>(&kb[r][l * 4]) = w;
     }
     __syncthreads();
-    float s[kCh / 4];
+    float acc[4][2];
 #pragma unroll
-    for (int u = 0; u < kCh / 4; ++u) s[u] = 0.f;
-    const float4* qa = reinterpret_cast<const float4*>(qs[qi]);
+    for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.f;
 #pragma unroll 4
     for (int x4 = 0; x4 < D / 4; ++x4) {
-      const float4 a = qa[x4];
+      float4 qv[4], kv[2];
 #pragma unroll
-      for (int u = 0; u < kCh / 4; ++u) {
-        const float4 w = reinterpret_cast<const float4*>(kb[part + 4 * u])[x4];
-        s[u] = fmaf(a.x, w.x, s[u]);
-        s[u] = fmaf(a.y, w.y, s[u]);
-        s[u] = fmaf(a.z, w.z, s[u]);
-        s[u] = fmaf(a.w, w.w, s[u]);
-      }
+      for (int i = 0; i < 4; ++i) qv[i] = reinterpret_cast<const float4*>(qs[ty + 16 * i])[x4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) kv[j] = reinterpret_cast<const float4*>(kb[tx + 16 * j])[x4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          acc[i][j] = fmaf(qv[i].x, kv[j].x, acc[i][j]);
+          acc[i][j] = fmaf(qv[i].y, kv[j].y, acc[i][j]);
+          acc[i][j] = fmaf(qv[i].z, kv[j].z, acc[i][j]);
+          acc[i][j] = fmaf(qv[i].w, kv[j].w, acc[i][j]);
+        }
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) sc[ty + 16 * i][tx + 16 * j] = acc[i][j];
+    __syncthreads();
 #pragma unroll
     for (int u = 0; u < kCh / 4; ++u) {
       const int jj = part + 4 * u;
       const int i = base + jj;
-      if (jj < nblk && i < c) insert<KM>(ts, ti, s[u], i);
+      if (jj < nblk && i < c) insert<KM>(ts, ti, sc[qi][jj], i);
     }
   }
 
@@ -176,8 +195,12 @@ template <typename T, int D, int KM>
 cudaError_t run(const Dims& dm, const void* q, const float* kbar, const int32_t* cu, int32_t* idx,
                 int* status, cudaStream_t st) {
   dim3 grid((dm.max_seqlen + kQ - 1) / kQ, dm.batch, dm.Hq);
-  gate_kernel<T, D, KM><<<grid, kThreads, 0, st>>>(dm, static_cast<const T*>(q), kbar, cu, idx,
-                                                   status);
+  const size_t smem = sizeof(float) * ((kQ + kCh) * (D + 4) + kQ * (kCh + 1));
+  cudaError_t e = cudaFuncSetAttribute(gate_kernel<T, D, KM>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  gate_kernel<T, D, KM><<<grid, kThreads, smem, st>>>(dm, static_cast<const T*>(q), kbar, cu,
+                                                      idx, status);
   return cudaGetLastError();
 }
 

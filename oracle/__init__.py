@@ -31,7 +31,7 @@ def _lib():
             "oracle_meanpool": [P, I, P, I, I, I, I, I, P],
             "oracle_gate_topk": [P, P, I, P, I, I, I, I, I, I, P, P],
             "oracle_forward": [P, P, P, I, P, I, I, I, I, I, I, P, P, P, P, P],
-            "oracle_forward_rows": [P, P, P, I, P, I, I, I, I, I, I, P, L, P, P, P, P, P],
+            "oracle_forward_rows": [P, P, P, I, P, I, I, I, I, I, I, P, L, P, P, P, P, P, P],
             "oracle_forward_mask": [P, P, P, I, P, I, I, I, I, I, I, P, P],
             "oracle_forward_two_branch": [P, P, P, I, P, I, I, I, I, I, I, I, P],
             "oracle_dense_causal": [P, P, P, I, P, I, I, I, I, P, P],
@@ -147,11 +147,26 @@ def forward(q, k, v, cu_seqlens, block_size, topk, indices=None):
     return out, lse, idx, nkeys
 
 
-def forward_rows(q, k, v, cu_seqlens, block_size, topk, rows, indices=None):
-    """Sampled forward on rows (row = t*Hq + h): (out [n,d], lse [n], idx [n,topk], gap [n])."""
-    qr, kr, vr, dt = _qkv(q, k, v)
+def forward_rows(q, k, v, cu_seqlens, block_size, topk, rows, indices=None, q_rows=None,
+                 num_q_heads=None):
+    """Sampled forward on rows (row = t*Hq + h): (out [n,d], lse [n], idx [n,topk], gap [n]).
+
+    With q_rows ([n, d], the q vectors of the listed rows) q may be None and
+    num_q_heads gives Hq; then the caller need not hold all of q."""
+    if q_rows is not None:
+        qr, dt = _raw(q_rows)
+        kr, dk = _raw(k)
+        vr, dv = _raw(v)
+        if not (dt == dk == dv):
+            raise TypeError("q_rows, k, v must share one dtype")
+        Hq, d = int(num_q_heads), qr.shape[-1]
+        T = kr.shape[0]
+        qbase = None
+    else:
+        qr, kr, vr, dt = _qkv(q, k, v)
+        T, Hq, d = qr.shape
+        qbase = qr
     cu = _i32(cu_seqlens)
-    T, Hq, d = qr.shape
     Hkv = kr.shape[1]
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
     n = len(rows)
@@ -160,9 +175,10 @@ def forward_rows(q, k, v, cu_seqlens, block_size, topk, rows, indices=None):
     lse = np.zeros(n, dtype=np.float64)
     idx = np.full((n, topk), -1, dtype=np.int32)
     gap = np.zeros(n, dtype=np.float64)
-    rc = _lib().oracle_forward_rows(_ptr(qr), _ptr(kr), _ptr(vr), dt, _ptr(cu), len(cu) - 1, Hq,
-                                    Hkv, d, block_size, topk, _ptr(rows), n, _ptr(idx_in),
-                                    _ptr(out), _ptr(lse), _ptr(idx), _ptr(gap))
+    rc = _lib().oracle_forward_rows(_ptr(qbase), _ptr(kr), _ptr(vr), dt, _ptr(cu), len(cu) - 1,
+                                    Hq, Hkv, d, block_size, topk, _ptr(rows), n, _ptr(idx_in),
+                                    _ptr(out), _ptr(lse), _ptr(idx), _ptr(gap),
+                                    _ptr(qr) if q_rows is not None else None)
     if rc:
         raise ValueError("oracle_forward_rows: invalid arguments")
     return out, lse, idx, gap

@@ -145,8 +145,10 @@ void select_blocks(const Problem& P, int64_t t, int h, int64_t p, const std::vec
 // chosen blocks: [PT §1 eq.4] with the current block causal [PT §2 eq.5].
 // Entries of sel that are not in [0, c) are not history blocks; block c is
 // always attended up to position p. Returns the number of keys attended.
-int64_t attend(const Problem& P, int b, int64_t t, int h, int64_t p, const int32_t* sel, double* o,
-               double* lse) {
+// The query vector is read from Pq at (tq, hq): P itself, or a one-row view
+// of the sampled q rows (oracle_forward_rows with q_rows).
+int64_t attend_q(const Problem& P, const Problem& Pq, int b, int64_t t, int h, int64_t tq, int hq,
+                 int64_t p, const int32_t* sel, double* o, double* lse) {
   const int64_t start = P.cu[b];
   const int g = h / (P.Hq / P.Hkv);
   const int64_t c = p / P.B;
@@ -167,7 +169,7 @@ int64_t attend(const Problem& P, int b, int64_t t, int h, int64_t p, const int32
   for (size_t r = 0; r < J.size(); ++r) {
     double acc = 0.0;
     for (int x = 0; x < P.d; ++x)
-      acc += load(P.q, P.dtype, q_off(P, t, h) + x) *
+      acc += load(Pq.q, P.dtype, q_off(Pq, tq, hq) + x) *
              load(P.k, P.dtype, kv_off(P, start + J[r], g) + x);
     logit[r] = acc * scale;
     m = std::max(m, logit[r]);
@@ -182,6 +184,11 @@ int64_t attend(const Problem& P, int b, int64_t t, int h, int64_t p, const int32
   for (int x = 0; x < P.d; ++x) o[x] /= l;
   if (lse) *lse = m + std::log(l);
   return static_cast<int64_t>(J.size());
+}
+
+int64_t attend(const Problem& P, int b, int64_t t, int h, int64_t p, const int32_t* sel, double* o,
+               double* lse) {
+  return attend_q(P, P, b, t, h, t, h, p, sel, o, lse);
 }
 
 // Sequence index of token t.
@@ -274,10 +281,12 @@ int oracle_forward(const void* q, const void* k, const void* v, int dtype, const
 
 // Sampled forward: only the rows listed (row = t * Hq + h). Per row it
 // writes out [nrows][d], lse [nrows], idx [nrows][topk], gap [nrows].
+// If q_rows is non-null it holds the q vectors of the listed rows ([nrows][d],
+// same dtype) and q is not read, so a caller need not hold all of q.
 int oracle_forward_rows(const void* q, const void* k, const void* v, int dtype, const int32_t* cu,
                         int batch, int Hq, int Hkv, int d, int B, int topk, const int64_t* rows,
                         int64_t nrows, const int32_t* idx_in, double* out, double* lse,
-                        int32_t* idx_out, double* gap) {
+                        int32_t* idx_out, double* gap, const void* q_rows) {
   Problem P{q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk};
   if (check(P)) return -1;
   const int64_t T = batch > 0 ? cu[batch] : 0;
@@ -303,15 +312,27 @@ int oracle_forward_rows(const void* q, const void* k, const void* v, int dtype, 
     const int h = static_cast<int>(rows[r] % Hq);
     const int b = seq_of(P, t);
     const int64_t p = t - cu[b];
+    // With q_rows, view row r as token 0 / head 0 of a one-row q array.
+    Problem Pr = P;
+    int64_t tq = t;
+    int hq = h;
+    if (q_rows) {
+      Pr.q = static_cast<const char*>(q_rows) +
+             r * static_cast<int64_t>(d) * (dtype == kBF16 ? 2 : 4);
+      Pr.Hq = 1;
+      tq = 0;
+      hq = 0;
+    }
     std::vector<int32_t> sel(static_cast<size_t>(topk));
     double gp = std::numeric_limits<double>::infinity();
     if (idx_in)
       std::memcpy(sel.data(), idx_in + r * topk, sizeof(int32_t) * topk);
     else
-      select_blocks(P, t, h, p, means[static_cast<size_t>(b) * Hkv + h / grp], sel.data(), &gp);
+      select_blocks(Pr, tq, hq, p, means[static_cast<size_t>(b) * Hkv + h / grp], sel.data(),
+                      &gp);
     if (idx_out) std::memcpy(idx_out + r * topk, sel.data(), sizeof(int32_t) * topk);
     if (gap) gap[r] = gp;
-    attend(P, b, t, h, p, sel.data(), out + r * d, lse ? lse + r : nullptr);
+    attend_q(P, Pr, b, t, h, tq, hq, p, sel.data(), out + r * d, lse ? lse + r : nullptr);
   }
   return 0;
 }

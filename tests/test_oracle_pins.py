@@ -347,3 +347,14 @@ def test_rows_mode_matches_full():
     assert (o == out.reshape(T * Hq, -1)[rows]).all()
     assert (i == idx.reshape(T * Hq, -1)[rows]).all()
     assert (l == lse.reshape(-1)[rows]).all()
+
+
+def test_rows_mode_with_only_the_sampled_q_rows():
+    lengths, B, topk = (64, 40), 8, 3
+    q, k, v, cu = small_case(lengths, 4, 2, 8, B, topk, dtype=torch.bfloat16, seed=15)
+    rows = np.array([3, 99, 250, 300])
+    full = oracle.forward_rows(q, k, v, cu, B, topk, rows)
+    q_rows = q.reshape(-1, 8)[torch.as_tensor(rows)]
+    part = oracle.forward_rows(None, k, v, cu, B, topk, rows, q_rows=q_rows, num_q_heads=4)
+    for a, b in zip(full, part):
+        assert (a == b).all()
