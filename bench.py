@@ -377,7 +377,9 @@ def main():
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     traffic = profile_traffic(os.path.join(ROOT, "long_context_prefill_block_b200", "csrc",
                                            "attn_tc.cu"), w.name)
-    launches_per_step = 2 + 7 * n_pass
+    tc_path = w.dtype == torch.bfloat16 and w.head_dim == 128 and w.block_size % 128 == 0
+    # mean-pool, gate; per pass: 4 regroup kernels, history, own-block (+ merge on the SIMT path)
+    launches_per_step = 2 + (6 if tc_path else 7) * n_pass
 
     if rank != 0:
         if world > 1:

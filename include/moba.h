@@ -137,8 +137,9 @@ MOBA_API int moba_num_passes(const moba_params* p);
  * caller, passed as void*). events[0] is recorded before the first launch,
  * events[1] after the mean-pool, events[2] after the gate/top-k, and for pass
  * j events[3+4j], [4+4j], [5+4j], [6+4j] after the regrouping, the history
- * attention, the own-block attention and the merge. Results are identical to
- * moba_forward. */
+ * attention, the own-block attention and the merge (on the tensor-core path
+ * the own-block kernel performs the merge, so the last interval is empty).
+ * Results are identical to moba_forward. */
 MOBA_API moba_status moba_forward_staged(const moba_params* p, const void* q, const void* k,
                                          const void* v, const int32_t* cu_seqlens, void* out,
                                          float* lse, void* ws, size_t ws_bytes,

@@ -17,7 +17,8 @@ cudaError_t launch_history_tc(const Dims& dm, const Chunk& ch, const void* q, co
                               const Partials& pt, int* status, cudaStream_t st);
 cudaError_t launch_current_tc(const Dims& dm, const Chunk& ch, const void* q, const void* k,
                               const void* v, const int32_t* cu, const int32_t* idx,
-                              const Partials& pt, int* status, cudaStream_t st);
+                              const Partials& pt, void* out, float* lse, int* status,
+                              cudaStream_t st);
 cudaError_t launch_dense_tc(const Dims& dm, const void* q, const void* k, const void* v,
                             const int32_t* cu, void* out, float* lse, int* status,
                             cudaStream_t st);
@@ -183,16 +184,18 @@ moba_status forward_impl(const moba_params* p, const void* q, const void* k, con
     MOBA_TRY(launch_regroup(dm, ch, idx, cu, rg, status, st));
     MOBA_TRY(mark());
     if (tc) {
+      // the own-block kernel merges the partials in its epilogue
       MOBA_TRY(launch_history_tc(dm, ch, q, k, v, cu, rg, pt, status, st));
       MOBA_TRY(mark());
-      MOBA_TRY(launch_current_tc(dm, ch, q, k, v, cu, idx, pt, status, st));
+      MOBA_TRY(launch_current_tc(dm, ch, q, k, v, cu, idx, pt, out, lse, status, st));
+      MOBA_TRY(mark());
     } else {
       MOBA_TRY(launch_history_simt(dm, ch, q, k, v, cu, rg, pt, st));
       MOBA_TRY(mark());
       MOBA_TRY(launch_current_simt(dm, ch, q, k, v, cu, idx, pt, st));
+      MOBA_TRY(mark());
+      MOBA_TRY(launch_merge(dm, ch, idx, cu, pt, out, lse, st));
     }
-    MOBA_TRY(mark());
-    MOBA_TRY(launch_merge(dm, ch, idx, cu, pt, out, lse, st));
     MOBA_TRY(mark());
   }
   return MOBA_OK;

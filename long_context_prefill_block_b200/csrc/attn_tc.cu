@@ -6,10 +6,12 @@
 //           chose the same earlier block, against that block's B raw keys,
 //           non-causal (eq. 6); writes a normalised partial result per slot;
 //   CUR   : 128 consecutive queries of one head against their own block,
-//           causal on the diagonal tile (eq. 5); writes a partial result;
+//           causal on the diagonal tile (eq. 5); its epilogue merges the
+//           result with the rows' history partials (eq. 7-8) and writes
+//           the output;
 //   DENSE : 128 consecutive queries against every earlier key of their
 //           sequence (eq. 1, causal); writes the output.
-// The partials are combined by the merge kernel with eq. (7)-(8).
+// HIST runs first; CUR then finds every history partial of its rows ready.
 //
 // Persistent CTAs (one per SM) walk a static list of 128-row query tiles.
 // Everything that a tile boundary would otherwise serialise is double
@@ -468,74 +470,148 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
       // Rows go out through a per-warp staging area so that every global
       // store instruction writes whole 128-byte segments of 4 or 8 rows.
       const uint32_t stage = sbase + kStageOff + (warp - 2) * 32 * kStageRow;
-      const int64_t orow = R.valid ? (MODE == DENSE ? R.t * dm.Hq + R.h : R.prow) : -1;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(tO + c * 32, rr);
-        tmem_wait_ld();
-        if (MODE == DENSE) {
+      if (MODE == CUR) {
+        // Own block done: merge with this row's history partials right here
+        // (eq. 7-8 written with lse: w_j = exp(lse_j - m), o = sum_j w_j o_j /
+        // sum_j w_j) and write the output; the own result never leaves the
+        // SM. Slots 0..slot-1 of the row hold the history partials. Each
+        // thread merges its own row with 32 independent 16-byte loads per
+        // slot in flight; the bf16 row then leaves through the staging area
+        // in whole 64-byte pieces.
+        const int slot = R.valid ? (int)(R.prow % dm.topk) : 0;
+        const int64_t prow0 = R.valid ? R.prow - slot : 0;
+        const int64_t orow = R.valid ? R.t * dm.Hq + R.h : -1;
+        float o[D];
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const uint32_t w0 = pack_bf16x2(__uint_as_float(rr[8 * x]) * inv_l,
-                                            __uint_as_float(rr[8 * x + 1]) * inv_l);
-            const uint32_t w1 = pack_bf16x2(__uint_as_float(rr[8 * x + 2]) * inv_l,
-                                            __uint_as_float(rr[8 * x + 3]) * inv_l);
-            const uint32_t w2 = pack_bf16x2(__uint_as_float(rr[8 * x + 4]) * inv_l,
-                                            __uint_as_float(rr[8 * x + 5]) * inv_l);
-            const uint32_t w3 = pack_bf16x2(__uint_as_float(rr[8 * x + 6]) * inv_l,
-                                            __uint_as_float(rr[8 * x + 7]) * inv_l);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(tO + c * 32, rr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[c * 32 + x] = __uint_as_float(rr[x]) * inv_l;
+        }
+        if (R.valid) {
+          float m = lse;
+          for (int j = 0; j < slot; ++j) m = fmaxf(m, a.part_lse[prow0 + j]);
+          const float w_own = ex2((lse - m) * 1.4426950408889634f);
+          float L = w_own;
+#pragma unroll
+          for (int x = 0; x < D; ++x) o[x] *= w_own;
+          for (int j = 0; j < slot; ++j) {
+            const float wj = ex2((a.part_lse[prow0 + j] - m) * 1.4426950408889634f);
+            L += wj;
+            const float4* src = reinterpret_cast<const float4*>(a.part_o + (prow0 + j) * D);
+#pragma unroll
+            for (int x4 = 0; x4 < D / 4; ++x4) {
+              const float4 v = src[x4];
+              o[4 * x4] = fmaf(wj, v.x, o[4 * x4]);
+              o[4 * x4 + 1] = fmaf(wj, v.y, o[4 * x4 + 1]);
+              o[4 * x4 + 2] = fmaf(wj, v.z, o[4 * x4 + 2]);
+              o[4 * x4 + 3] = fmaf(wj, v.w, o[4 * x4 + 3]);
+            }
+          }
+          const float inv = 1.f / L;
+#pragma unroll
+          for (int x = 0; x < D; ++x) o[x] *= inv;
+          if (a.lse_out) a.lse_out[orow] = m + logf(L);
+        }
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
                              stage + lane * 80 + x * 16),
-                         "r"(w0), "r"(w1), "r"(w2), "r"(w3)
+                         "r"(pack_bf16x2(o[c * 32 + 8 * x], o[c * 32 + 8 * x + 1])),
+                         "r"(pack_bf16x2(o[c * 32 + 8 * x + 2], o[c * 32 + 8 * x + 3])),
+                         "r"(pack_bf16x2(o[c * 32 + 8 * x + 4], o[c * 32 + 8 * x + 5])),
+                         "r"(pack_bf16x2(o[c * 32 + 8 * x + 6], o[c * 32 + 8 * x + 7]))
                          : "memory");
-          }
           __syncwarp();
           // 64 bytes per row chunk: 4 lanes per row, 8 rows per instruction
 #pragma unroll
           for (int it = 0; it < 4; ++it) {
             const int row = it * 8 + (lane >> 2), seg = lane & 3;
-            const int64_t o = __shfl_sync(0xffffffffu, orow, row);
+            const int64_t orr = __shfl_sync(0xffffffffu, orow, row);
             uint4 val;
             asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
                          : "r"(stage + row * 80 + seg * 16)
                          : "memory");
-            if (o >= 0)
-              *reinterpret_cast<uint4*>(a.out + o * D + c * 32 + seg * 8) = val;
+            if (orr >= 0)
+              *reinterpret_cast<uint4*>(a.out + orr * D + c * 32 + seg * 8) = val;
           }
-        } else {
-#pragma unroll
-          for (int x = 0; x < 8; ++x)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                             stage + lane * kStageRow + x * 16),
-                         "r"(__float_as_uint(__uint_as_float(rr[4 * x]) * inv_l)),
-                         "r"(__float_as_uint(__uint_as_float(rr[4 * x + 1]) * inv_l)),
-                         "r"(__float_as_uint(__uint_as_float(rr[4 * x + 2]) * inv_l)),
-                         "r"(__float_as_uint(__uint_as_float(rr[4 * x + 3]) * inv_l))
-                         : "memory");
           __syncwarp();
-          // 128 bytes per row chunk: 8 lanes per row, 4 rows per instruction
-#pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int row = it * 4 + (lane >> 3), seg = lane & 7;
-            const int64_t o = __shfl_sync(0xffffffffu, orow, row);
-            uint4 val;
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                         : "r"(stage + row * kStageRow + seg * 16)
-                         : "memory");
-            if (o >= 0)
-              *reinterpret_cast<uint4*>(a.part_o + o * D + c * 32 + seg * 4) = val;
-          }
         }
-        __syncwarp();
-      }
-      if (R.valid) {
-        if (MODE == DENSE) {
-          if (a.lse_out) a.lse_out[R.t * dm.Hq + R.h] = lse;
-        } else {
-          a.part_lse[R.prow] = lse;
+      } else {
+        const int64_t orow = R.valid ? (MODE == DENSE ? R.t * dm.Hq + R.h : R.prow) : -1;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(tO + c * 32, rr);
+          tmem_wait_ld();
+          if (MODE == DENSE) {
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              const uint32_t w0 = pack_bf16x2(__uint_as_float(rr[8 * x]) * inv_l,
+                                              __uint_as_float(rr[8 * x + 1]) * inv_l);
+              const uint32_t w1 = pack_bf16x2(__uint_as_float(rr[8 * x + 2]) * inv_l,
+                                              __uint_as_float(rr[8 * x + 3]) * inv_l);
+              const uint32_t w2 = pack_bf16x2(__uint_as_float(rr[8 * x + 4]) * inv_l,
+                                              __uint_as_float(rr[8 * x + 5]) * inv_l);
+              const uint32_t w3 = pack_bf16x2(__uint_as_float(rr[8 * x + 6]) * inv_l,
+                                              __uint_as_float(rr[8 * x + 7]) * inv_l);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                               stage + lane * 80 + x * 16),
+                           "r"(w0), "r"(w1), "r"(w2), "r"(w3)
+                           : "memory");
+            }
+            __syncwarp();
+            // 64 bytes per row chunk: 4 lanes per row, 8 rows per instruction
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int row = it * 8 + (lane >> 2), seg = lane & 3;
+              const int64_t o = __shfl_sync(0xffffffffu, orow, row);
+              uint4 val;
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                           : "r"(stage + row * 80 + seg * 16)
+                           : "memory");
+              if (o >= 0)
+                *reinterpret_cast<uint4*>(a.out + o * D + c * 32 + seg * 8) = val;
+            }
+          } else {
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                               stage + lane * kStageRow + x * 16),
+                           "r"(__float_as_uint(__uint_as_float(rr[4 * x]) * inv_l)),
+                           "r"(__float_as_uint(__uint_as_float(rr[4 * x + 1]) * inv_l)),
+                           "r"(__float_as_uint(__uint_as_float(rr[4 * x + 2]) * inv_l)),
+                           "r"(__float_as_uint(__uint_as_float(rr[4 * x + 3]) * inv_l))
+                           : "memory");
+            __syncwarp();
+            // 128 bytes per row chunk: 8 lanes per row, 4 rows per instruction
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+              const int row = it * 4 + (lane >> 3), seg = lane & 7;
+              const int64_t o = __shfl_sync(0xffffffffu, orow, row);
+              uint4 val;
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                           : "r"(stage + row * kStageRow + seg * 16)
+                           : "memory");
+              if (o >= 0)
+                *reinterpret_cast<uint4*>(a.part_o + o * D + c * 32 + seg * 4) = val;
+            }
+          }
+          __syncwarp();
+        }
+        if (R.valid) {
+          if (MODE == DENSE) {
+            if (a.lse_out) a.lse_out[R.t * dm.Hq + R.h] = lse;
+          } else {
+            a.part_lse[R.prow] = lse;
+          }
         }
       }
       fence_before_sync();
@@ -662,12 +738,15 @@ cudaError_t launch_history_tc(const Dims& dm, const Chunk& ch, const void* q, co
 
 cudaError_t launch_current_tc(const Dims& dm, const Chunk& ch, const void* q, const void* k,
                               const void* v, const int32_t* cu, const int32_t* idx,
-                              const Partials& pt, int* status, cudaStream_t st) {
+                              const Partials& pt, void* out, float* lse, int* status,
+                              cudaStream_t st) {
   if (dm.batch == 0 || dm.max_seqlen == 0) return cudaSuccess;
   Args a = base_args(dm, ch, q, cu, status);
   a.idx = idx;
   a.part_o = pt.o;
   a.part_lse = pt.lse;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse_out = lse;
   const int64_t tiles = (int64_t)(dm.B / TM) * dm.nb * dm.batch * ch.nq;
   a.n_tiles = (int)tiles;
   return launch<CUR>(tiles, a, k, v, st);

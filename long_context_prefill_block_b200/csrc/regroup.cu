@@ -78,6 +78,65 @@ __global__ void __launch_bounds__(kThreads) regroup_pass(Dims dm, Chunk ch,
   if (!SCATTER && !ok) set_status(status, kStBadIndices);
 }
 
+// Same two passes with the lists of one CTA (kRows positions of one q head,
+// hence one sequence and kv head) counted in shared memory first, so each
+// list sees one global atomic per CTA instead of one per entry. The scatter
+// pass reserves a contiguous range per list and places the CTA's entries in
+// it. Used when a sequence has at most kSmemLists blocks.
+constexpr int kRows = 256;
+constexpr int kSmemLists = 8192;
+
+template <bool SCATTER>
+__global__ void __launch_bounds__(kRows) regroup_pass_smem(Dims dm, Chunk ch,
+                                                           const int32_t* __restrict__ idx,
+                                                           const int32_t* __restrict__ cu,
+                                                           int32_t* counts, int32_t* cursor,
+                                                           const int32_t* __restrict__ list_off,
+                                                           int32_t* pairs, int* status) {
+  extern __shared__ int32_t lsm[];
+  int32_t* hist = lsm;            // [nb] entries of this CTA per block
+  int32_t* base = lsm + dm.nb;    // [nb] SCATTER: first list position reserved for the CTA
+  const int b = blockIdx.y, hl = blockIdx.z;
+  const int h = ch.h0 + hl;
+  const int grp = dm.Hq / dm.Hkv;
+  const int gl = h / grp - ch.g0;
+  int64_t start;
+  int len;
+  if (!seq_bounds(dm, cu, b, start, len, SCATTER ? nullptr : status)) return;
+  const int p0 = blockIdx.x * kRows;
+  if (p0 >= len) return;
+  const int cmax = (min(p0 + kRows, len) - 1) / dm.B + 1;  // blocks any row may name
+  for (int e = threadIdx.x; e < cmax; e += kRows) hist[e] = 0;
+  __syncthreads();
+  const int p = p0 + threadIdx.x;
+  const bool valid = p < len;
+  const int64_t t = start + p;
+  const int c = p / dm.B;
+  const int32_t* row = idx + (t * dm.Hq + h) * (int64_t)dm.topk;
+  const int list0 = (b * ch.ng + gl) * dm.nb;
+  const int64_t prow0 = (t * ch.nq + hl) * (int64_t)dm.topk;
+  bool ok = true;
+  if (valid) ok = walk_row(row, dm.topk, c, [&](int, int e) { atomicAdd(&hist[e], 1); });
+  if (!SCATTER && !ok) set_status(status, kStBadIndices);
+  __syncthreads();
+  for (int e = threadIdx.x; e < cmax; e += kRows) {
+    const int n = hist[e];
+    if (SCATTER) {
+      base[e] = n ? atomicAdd(&cursor[list0 + e], n) : 0;
+      hist[e] = 0;
+    } else if (n) {
+      atomicAdd(&counts[list0 + e], n);
+    }
+  }
+  if (!SCATTER) return;
+  __syncthreads();
+  if (valid)
+    walk_row(row, dm.topk, c, [&](int slot, int e) {
+      const int pos = base[e] + atomicAdd(&hist[e], 1);
+      pairs[list_off[list0 + e] + pos] = (int32_t)(prow0 + slot);
+    });
+}
+
 // Exclusive scans of the list sizes and of their tile counts (one CTA).
 __global__ void __launch_bounds__(kScanThreads) regroup_scan(int n_lists, int tile_m,
                                                             const int32_t* __restrict__ counts,
@@ -160,15 +219,34 @@ cudaError_t launch_regroup(const Dims& dm, const Chunk& ch, const int32_t* idx, 
   if (dm.batch == 0 || dm.max_seqlen == 0) {
     return cudaMemsetAsync(rg.tile_off + ch.n_lists, 0, sizeof(int32_t), st);
   }
+  const bool smem_lists = dm.nb <= kSmemLists;
   dim3 grid((dm.max_seqlen + kThreads - 1) / kThreads, dm.batch, ch.nq);
-  regroup_pass<false><<<grid, kThreads, 0, st>>>(dm, ch, idx, cu, rg.counts, rg.cursor, nullptr,
-                                                 nullptr, status);
+  dim3 grid_s((dm.max_seqlen + kRows - 1) / kRows, dm.batch, ch.nq);
+  const size_t lsm = 2 * sizeof(int32_t) * dm.nb;
+  if (smem_lists) {
+    if ((e = cudaFuncSetAttribute(regroup_pass_smem<false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsm)))
+      return e;
+    if ((e = cudaFuncSetAttribute(regroup_pass_smem<true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsm)))
+      return e;
+    regroup_pass_smem<false><<<grid_s, kRows, lsm, st>>>(dm, ch, idx, cu, rg.counts, rg.cursor,
+                                                         nullptr, nullptr, status);
+  } else {
+    regroup_pass<false><<<grid, kThreads, 0, st>>>(dm, ch, idx, cu, rg.counts, rg.cursor, nullptr,
+                                                   nullptr, status);
+  }
   if ((e = cudaGetLastError())) return e;
   regroup_scan<<<1, kScanThreads, 0, st>>>(ch.n_lists, ch.tile_m, rg.counts, rg.list_off,
                                            rg.tile_off);
   if ((e = cudaGetLastError())) return e;
-  regroup_pass<true><<<grid, kThreads, 0, st>>>(dm, ch, idx, cu, rg.counts, rg.cursor, rg.list_off,
-                                                rg.pairs, status);
+  if (smem_lists) {
+    regroup_pass_smem<true><<<grid_s, kRows, lsm, st>>>(dm, ch, idx, cu, rg.counts, rg.cursor,
+                                                        rg.list_off, rg.pairs, status);
+  } else {
+    regroup_pass<true><<<grid, kThreads, 0, st>>>(dm, ch, idx, cu, rg.counts, rg.cursor,
+                                                  rg.list_off, rg.pairs, status);
+  }
   if ((e = cudaGetLastError())) return e;
   regroup_tiles<<<(ch.n_lists + 255) / 256, 256, 0, st>>>(ch.n_lists, ch.tile_m, rg.counts,
                                                           rg.tile_off, rg.tiles);
