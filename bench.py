@@ -71,6 +71,23 @@ def row_flops(w, rows):
     return int((4 * w.head_dim * nkeys).sum())
 
 
+def rank_workload(w, rank: int):
+    """Rank r of a weak-scaling run processes its own batch: same shapes, its
+    own seed (independent problems, no collective on the data path)."""
+    import dataclasses
+
+    return dataclasses.replace(w, seed=w.seed + 7919 * rank) if rank else w
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    """Max over ranks (slowest rank's time)."""
+    if world == 1:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -238,7 +255,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    q, k, v, cu = make_inputs(w, dev)
+    q, k, v, cu = make_inputs(rank_workload(w, rank), dev)
     cu_d = cu.to(dev)
     p = moba.make_params(q, k, cu, w.block_size, w.topk, w.max_seqlen)
     ws = moba.workspace(p, dev)
@@ -261,11 +278,7 @@ def main():
             torch.distributed.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     clocks = ClockSampler(dev.index) if rank == 0 else None
     if clocks:

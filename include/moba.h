@@ -170,6 +170,14 @@ MOBA_API moba_status dense_causal_forward(const moba_params* p, const void* q, c
  * if `clear` is non-zero. */
 MOBA_API moba_status moba_device_status(void* stream, int clear);
 
+/* Self-test of the bounded waits used by the tensor-core kernels (no paper
+ * counterpart; failure detection): launches one CTA that waits on a barrier
+ * nothing arrives on. After about 2e9 SM cycles (about a second) the wait
+ * gives up, the kernel writes 2 to *done (device int) and records
+ * MOBA_ERR_TIMEOUT in the status word, which moba_device_status() then
+ * returns; the context stays usable. Nothing faults or hangs. */
+MOBA_API moba_status moba_selftest_bounded_wait(int* done, void* stream);
+
 /* Static description of a status code. */
 MOBA_API const char* moba_status_string(moba_status s);
 

@@ -218,6 +218,18 @@ def dense_causal_forward(q, k, v, cu_seqlens, max_seqlen=None, return_lse: bool 
     return (out, lse) if return_lse else out
 
 
+def moba_selftest_bounded_wait(device=None) -> int:
+    """Run the bounded-wait self-test kernel; returns the kernel's verdict
+    (2 = the wait gave up as it must). Read moba_device_status() afterwards."""
+    fn = lib().moba_selftest_bounded_wait
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    done = torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+    _check("moba_selftest_bounded_wait", fn(_ptr(done), _stream(done.device)))
+    torch.cuda.synchronize(done.device)
+    return int(done.item())
+
+
 def moba_device_status(device=None, clear: bool = True) -> int:
     """Synchronise the current stream and return (and clear) the device status word."""
     return int(lib().moba_device_status(_stream(device), int(clear)))

@@ -23,6 +23,7 @@ cudaError_t launch_dense_tc(const Dims& dm, const void* q, const void* k, const 
                             const int32_t* cu, void* out, float* lse, int* status,
                             cudaStream_t st);
 bool tc_supported(const Dims& dm);
+cudaError_t launch_wait_selftest(int* status, int* done, cudaStream_t st);
 constexpr int kTcTileM = 128;
 }  // namespace moba
 
@@ -311,6 +312,13 @@ moba_status moba_device_status(void* stream, int clear) {
     if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return MOBA_ERR_CUDA;
   }
   return static_cast<moba_status>(value);
+}
+
+moba_status moba_selftest_bounded_wait(int* done, void* stream) {
+  if (!done) return MOBA_ERR_INVALID_ARG;
+  int* status = status_word();
+  if (!status) return MOBA_ERR_CUDA;
+  return cuda_status(launch_wait_selftest(status, done, static_cast<cudaStream_t>(stream)));
 }
 
 const char* moba_status_string(moba_status s) {
