@@ -24,7 +24,7 @@ cudaError_t launch_dense_tc(const Dims& dm, const void* q, const void* k, const 
                             cudaStream_t st);
 bool tc_supported(const Dims& dm);
 cudaError_t launch_wait_selftest(int* status, int* done, cudaStream_t st);
-constexpr int kTcTileM = 128;
+int tc_tile_m();
 }  // namespace moba
 
 using namespace moba;
@@ -81,7 +81,7 @@ Layout plan(const Dims& dm, bool own_idx) {
   L.ng = (int)ng;
   const int64_t n_lists = (int64_t)dm.batch * L.ng * dm.nb;
   const int64_t max_pairs = (int64_t)dm.T * L.ng * grp * (dm.topk - 1);
-  const int tile_m = kSimtTileM < kTcTileM ? kSimtTileM : kTcTileM;
+  const int tile_m = kSimtTileM < tc_tile_m() ? kSimtTileM : tc_tile_m();
   L.max_tiles = (max_pairs + tile_m - 1) / tile_m + n_lists;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -179,7 +179,7 @@ moba_status forward_impl(const moba_params* p, const void* q, const void* k, con
     ch.h0 = g0 * grp;
     ch.nq = ch.ng * grp;
     ch.n_lists = dm.batch * ch.ng * dm.nb;
-    ch.tile_m = tc ? kTcTileM : kSimtTileM;
+    ch.tile_m = tc ? tc_tile_m() : kSimtTileM;
     const int64_t pairs = (int64_t)dm.T * ch.nq * (dm.topk - 1);
     rg.max_tiles = (pairs + ch.tile_m - 1) / ch.tile_m + ch.n_lists;
     MOBA_TRY(launch_regroup(dm, ch, idx, cu, rg, status, st));

@@ -13,27 +13,31 @@
 //           sequence (eq. 1, causal); writes the output.
 // HIST runs first; CUR then finds every history partial of its rows ready.
 //
-// Persistent CTAs (one per SM) walk a static list of 128-row query tiles.
-// Everything that a tile boundary would otherwise serialise is double
-// buffered: the query tile in shared memory (Q[2]), the logits in TMEM
-// (S[2], 128 fp32 columns each) and the output accumulator in TMEM (O[2]),
-// so the next tile's Q gather and first QK^T overlap the current tile's last
-// softmax and epilogue. Roles (8 warps):
-//   warp 0     TMA producer: K and V tiles of 128 keys (two 64-column
-//              halves, 128-byte swizzle) into a 2-stage ring;
-//   warp 1     allocates all 512 TMEM columns; lane 0 issues every
-//              tcgen05.mma: S = Q K^T, then O += P V for the previous KV tile
-//              with P read from TMEM (bf16, packed into the first 64 columns
-//              of the S buffer it came from);
-//   warps 2-5  softmax + epilogue, one query row per thread (TMEM lane =
-//              row): base-2 exponentials, P store, running (m, l); O is
-//              rescaled only when a row maximum grows by more than 2^8, so
-//              PV normally never waits for the softmax warps;
-//   warps 6-7  Q loaders: cp.async of the tile's (gathered, in HIST mode)
-//              query rows straight into the swizzled layout the MMA reads.
-// KV tiles are numbered globally per CTA (g); S buffer g % 2, ring stage
-// g % 2 and every barrier phase follow from g, Q/O buffers from the tile
-// count i.
+// Persistent CTAs (one per SM) walk a static list of work units of two
+// 128-row query halves that read the same KV tiles (HIST: 256 consecutive
+// rows of one block's list; CUR / DENSE: two consecutive 128-row query
+// tiles, the second one seeing one more KV tile). Each KV tile (128 keys) is
+// loaded once and used by both halves, which halves the shared-memory fill
+// traffic per flop, and the two halves ping-pong on the tensor core: while
+// one half's softmax runs, the other half's MMAs do. TMEM holds per half h
+// the logits S[h] (128 fp32 columns; P overwrites its first 64 columns as
+// bf16 pairs) and the accumulator O[h]. Roles (12 warps):
+//   warp 0      TMA producer: K and V tiles of 128 keys (two 64-column
+//               halves, 128-byte swizzle) into a 2-stage ring;
+//   warps 1-2   lane 0 of warp 1 + h issues the tcgen05.mma of half h (warp
+//               1 also allocates all 512 TMEM columns): S[h] = Q_h K(0)^T,
+//               then per KV tile j O[h] += P_h(j) V(j) and S[h] = Q_h
+//               K(j+1)^T into the same TMEM -- tcgen05.mma operations of one
+//               thread run in issue order, so the PV has read P before the
+//               next QK^T overwrites it. Issuing blocks for about the
+//               group's execution time, hence one issuer per half;
+//   warp 3      Q loader: cp.async of each half's (gathered, in HIST mode)
+//               query rows into the swizzled layout the MMA reads;
+//   warps 4-7   softmax + epilogue of half 0, warps 8-11 of half 1: one query
+//               row per thread (TMEM lane = row), base-2 exponentials; O[h]
+//               is rescaled only when a row maximum grows by more than 2^8.
+// The softmax warps get most of the register file (setmaxnreg): they hold a
+// whole 128-column row of S, or of O in the epilogue.
 //
 // Every wait is bounded (tc::mbar_wait); on expiry the CTA records
 // kStTimeout, drains the copies and MMAs it issued, frees its TMEM and exits.
@@ -53,34 +57,40 @@ using namespace tc;
 
 enum Mode { HIST = 0, CUR = 1, DENSE = 2 };
 
-constexpr int TM = 128;   // query rows per tile
+constexpr int TM = 128;   // query rows per half
 constexpr int TN = 128;   // keys per KV tile
 constexpr int D = 128;    // head dim
 constexpr int NS = 2;     // K/V ring stages
-constexpr int kThreads = 256;
-constexpr int kLoaderThreads = 64;
+constexpr int kThreads = 384;
+constexpr int kLoaderThreads = 32;
+constexpr int kLaunchRegs = 168;    // 65536 / 384, rounded down to a multiple of 8
+constexpr int kRegsOther = 72;      // warps 0-3 after setmaxnreg.dec
+constexpr int kRegsSoftmax = 216;   // warps 4-11 after setmaxnreg.inc
+static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr uint32_t kHalf = 128 * 128;  // bytes of one 64-column half of a 128-row tile
 constexpr uint32_t kTile = 2 * kHalf;  // bytes of one 128 x 128 bf16 tile
-constexpr uint32_t kQOff = 0;          // Q[2]
+constexpr uint32_t kQOff = 0;          // Q[2], one per query half
 constexpr uint32_t kKOff = 2 * kTile;  // K[NS]
 constexpr uint32_t kVOff = kKOff + NS * kTile;
-constexpr uint32_t kStageRow = 144;    // bytes per staged row: 32 fp32 + 16 pad
+constexpr uint32_t kStageRow = 80;     // bytes per staged row chunk: 64 + 16 pad
 constexpr uint32_t kStageOff = kVOff + NS * kTile;  // epilogue staging, 32 rows per softmax warp
-constexpr uint32_t kStageBytes = 4 * 32 * kStageRow;
+constexpr uint32_t kStageBytes = 8 * 32 * kStageRow;
 constexpr uint32_t kSmemBytes = kStageOff + kStageBytes + 1024;  // + 1024-byte alignment slack
 constexpr uint32_t kTmemCols = 512;    // S[0] 0, S[1] 128, O[0] 256, O[1] 384
+constexpr uint32_t kOCol = 256;
 constexpr uint32_t kIdescQK = idesc_bf16(TM, TN, false, false);  // Q, K both K-major
 constexpr uint32_t kIdescPV = idesc_bf16(TM, D, false, true);    // V is MN-major (d contiguous)
 constexpr float kRescaleLog2 = 8.f;
 
 struct Shared {
-  uint64_t q_full[2], q_empty[2];
+  // per query half h
+  uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_free[2];
   uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
-  uint64_t s_full[2], s_free[2], p_full[2];
-  uint64_t o_full[2], o_free[2];
-  uint64_t drain;
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
+  int exp_cnt[2];  // per half: softmax warps done with a KV tile's exponentials
 };
 
 struct Args {
@@ -104,13 +114,17 @@ struct Args {
   int* status;
 };
 
+// A work unit: half 0 is described by the fields below; half 1 starts 128
+// rows later (half_view). n[h] = KV tiles half h reads (0: half h is empty);
+// the unit streams max(n[0], n[1]) KV tiles.
 struct Tile {
   bool skip;
   int b, g, h, kv0, n_kv, p0, list, row0, count;
+  int n[2];
   int64_t start;
 };
 
-// Tile t of the static tile space. CUR / DENSE tiles are ordered longest
+// Unit t of the static unit space. CUR / DENSE units are ordered longest
 // first so the persistent CTAs end together.
 template <int MODE>
 __device__ __forceinline__ Tile get_tile(const Args& a, int t) {
@@ -127,40 +141,58 @@ __device__ __forceinline__ Tile get_tile(const Args& a, int t) {
     T.count = a.list_off[T.list + 1] - a.list_off[T.list];
     T.kv0 = e * dm.B;
     T.n_kv = dm.B / TN;
+    T.n[0] = T.n_kv;
+    T.n[1] = T.row0 + TM < T.count ? T.n_kv : 0;
     T.start = a.cu[T.b];
     return T;
   }
-  int qt;
+  int m;  // the unit holds query tiles 2m and 2m + 1 (of the block / sequence)
   if (MODE == CUR) {
     const int R = dm.B / TM;                      // query tiles per block
-    const int per = dm.nb * dm.batch * a.ch.nq;   // tiles with the same r
-    const int r = R - 1 - t / per;
+    const int R2 = (R + 1) / 2;                   // units per block
+    const int per = dm.nb * dm.batch * a.ch.nq;   // units with the same m
+    m = R2 - 1 - t / per;
     int rem = t % per;
     const int c = rem / (dm.batch * a.ch.nq);
     rem %= dm.batch * a.ch.nq;
     T.b = rem / a.ch.nq;
     T.h = a.ch.h0 + rem % a.ch.nq;
-    T.p0 = c * dm.B + r * TM;
+    T.p0 = c * dm.B + 2 * m * TM;
     T.kv0 = c * dm.B;
-    T.n_kv = r + 1;
-    qt = 0;
+    T.n[1] = 2 * m + 1 < R ? 2 * m + 2 : 0;
   } else {
     const int nqt = (dm.max_seqlen + TM - 1) / TM;
+    const int nqt2 = (nqt + 1) / 2;
     const int per = dm.batch * dm.Hq;
-    qt = nqt - 1 - t / per;
+    m = nqt2 - 1 - t / per;
     const int rem = t % per;
     T.b = rem / dm.Hq;
     T.h = rem % dm.Hq;
-    T.p0 = qt * TM;
+    T.p0 = 2 * m * TM;
     T.kv0 = 0;
-    T.n_kv = qt + 1;
+    T.n[1] = 2 * m + 2;
   }
+  T.n[0] = 2 * m + 1;
   T.g = T.h / (dm.Hq / dm.Hkv);
   T.start = a.cu[T.b];
   const int len = a.cu[T.b + 1] - a.cu[T.b];
   T.count = len;  // sequence length, for the row checks below
   T.skip = len < 0 || len > dm.max_seqlen || T.p0 >= len;
+  if (T.p0 + TM >= len) T.n[1] = 0;
+  T.n_kv = T.n[1] > T.n[0] ? T.n[1] : T.n[0];
   return T;
+}
+
+// The tile of query half h of a unit, as the row helpers below see it.
+template <int MODE>
+__device__ __forceinline__ Tile half_view(const Tile& T, int h) {
+  Tile U = T;
+  if (MODE == HIST)
+    U.row0 += h * TM;
+  else
+    U.p0 += h * TM;
+  U.n_kv = T.n[h];
+  return U;
 }
 
 // Identity of query row r of a tile: the q row it reads (t * Hq + h, or -1)
@@ -217,6 +249,13 @@ __device__ __forceinline__ bool q_row_of(const Args& a, const Tile& T, int r, in
   return true;
 }
 
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+}
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -237,19 +276,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
       mbar_init(&sh.q_full[i], kLoaderThreads);
       mbar_init(&sh.q_empty[i], 1);
       mbar_init(&sh.s_full[i], 1);
-      mbar_init(&sh.s_free[i], 1);
       mbar_init(&sh.p_full[i], 128);
       mbar_init(&sh.o_full[i], 1);
       mbar_init(&sh.o_free[i], 128);
     }
     for (int i = 0; i < NS; ++i) {
       mbar_init(&sh.k_full[i], 1);
-      mbar_init(&sh.k_empty[i], 1);
+      mbar_init(&sh.k_empty[i], 2);  // one commit from each issuer
       mbar_init(&sh.v_full[i], 1);
-      mbar_init(&sh.v_empty[i], 1);
+      mbar_init(&sh.v_empty[i], 2);
     }
-    mbar_init(&sh.drain, 1);
+    mbar_init(&sh.drain[0], 1);
+    mbar_init(&sh.drain[1], 1);
     sh.abort = 0;
+    sh.exp_cnt[0] = sh.exp_cnt[1] = 0;
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -263,121 +303,174 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
   volatile int* abort = &sh.abort;
   int* status = a.status;
 
-  if (warp == 0) {
-    // ================= TMA producer: K and V tiles =================
-    if (lane == 0) {
-      uint32_t g = 0, nk = 0, nv = 0;
+  if (warp < 4) {
+    // warps 0-3 (one warp group) give registers to the softmax warps
+    regs_dec();
+    if (warp == 0) {
+      // ================= TMA producer: K and V tiles =================
+      if (lane == 0) {
+        uint32_t g = 0, nk = 0, nv = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+          const Tile T = get_tile<MODE>(a, t);
+          if (T.skip) continue;
+          for (int j = 0; j < T.n_kv; ++j, ++g) {
+            const uint32_t st = g % NS, u = g / NS;
+            const int z = (int)(T.start + T.kv0 + j * TN);
+            if (u > 0 && !(ok = mbar_wait(&sh.k_empty[st], (u - 1) & 1, abort, status))) break;
+            mbar_expect_tx(&sh.k_full[st], kTile);
+            tma_load_3d(sK + st * kTile, &tmk, &sh.k_full[st], 0, T.g, z);
+            tma_load_3d(sK + st * kTile + kHalf, &tmk, &sh.k_full[st], 64, T.g, z);
+            nk = g + 1;
+            if (u > 0 && !(ok = mbar_wait(&sh.v_empty[st], (u - 1) & 1, abort, status))) break;
+            mbar_expect_tx(&sh.v_full[st], kTile);
+            tma_load_3d(sV + st * kTile, &tmv, &sh.v_full[st], 0, T.g, z);
+            tma_load_3d(sV + st * kTile + kHalf, &tmv, &sh.v_full[st], 64, T.g, z);
+            nv = g + 1;
+          }
+        }
+        if (!ok || *abort) {
+          // let the copies already issued land before the CTA exits
+          for (uint32_t x = nk > NS ? nk - NS : 0; x < nk; ++x)
+            mbar_drain(&sh.k_full[x % NS], (x / NS) & 1);
+          for (uint32_t x = nv > NS ? nv - NS : 0; x < nv; ++x)
+            mbar_drain(&sh.v_full[x % NS], (x / NS) & 1);
+        }
+      }
+    } else if (warp < 3) {
+      // ====== MMA issuers: warp 1 for query half 0, warp 2 for half 1 ======
+      // One thread per half: issuing a group of MMAs blocks the thread for
+      // about the group's execution time, so a single issuer would make each
+      // half wait behind the other's groups. Per half the order is QK(0),
+      // then PV(j), QK(j + 1) for each KV tile j; K(j) and V(j) are
+      // released by both issuers (empty barriers count two), also for tiles
+      // a half skips.
+      const int h = warp - 1;
+      if (lane == 0) {
+        uint32_t gk = 0;  // KV tiles streamed before this unit
+        uint32_t kh = 0;  // KV tiles of this half before this unit
+        uint32_t uh = 0;  // units with this half non-empty before this one
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+          const Tile T = get_tile<MODE>(a, t);
+          if (T.skip) continue;
+          const int nh = T.n[h];
+          for (int j = 0; ok && j < T.n_kv; ++j) {
+            const uint32_t gg = gk + j, st = gg % NS;
+            // Both issuers wait for every tile, also one they skip, before
+            // releasing it: an early release could complete the barrier
+            // phase of an older tile that the other issuer still reads.
+            if (!(ok = mbar_wait(&sh.k_full[st], (gg / NS) & 1, abort, status))) break;
+            if (j < nh) {
+              // S[h] = Q_h K(j)^T; S[h] holds P(j - 1) until PV(j - 1), which
+              // this thread issued before
+              if (j == 0 && !(ok = mbar_wait(&sh.q_full[h], uh & 1, abort, status))) break;
+              fence_after_sync();
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+                const uint64_t ad = desc_sw128(sQ + h * kTile + off, 16, 1024);
+                const uint64_t bd = desc_sw128(sK + st * kTile + off, 16, 1024);
+                mma_ss(tmem + h * 128, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
+              }
+              commit(&sh.s_full[h]);
+              if (j == nh - 1) commit(&sh.q_empty[h]);
+            }
+            commit(&sh.k_empty[st]);
+            if (j < nh) {
+              // O[h] += P_h(j) V(j), P read from the first 64 columns of S[h]
+              if (j == 0 && uh > 0 &&
+                  !(ok = mbar_wait(&sh.o_free[h], (uh - 1) & 1, abort, status)))
+                break;
+              if (!(ok = mbar_wait(&sh.p_full[h], (kh + j) & 1, abort, status))) break;
+            }
+            if (!(ok = mbar_wait(&sh.v_full[st], (gg / NS) & 1, abort, status))) break;
+            if (j < nh) {
+              fence_after_sync();
+#pragma unroll
+              for (int kk = 0; kk < TN / 16; ++kk) {
+                const uint64_t bd = desc_sw128(sV + st * kTile + kk * 16 * 128, kHalf, 1024);
+                mma_ts(tmem + kOCol + h * 128, tmem + h * 128 + kk * 8, bd, kIdescPV,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+              }
+              if (j == nh - 1) commit(&sh.o_full[h]);
+            }
+            commit(&sh.v_empty[st]);
+          }
+          gk += T.n_kv;
+          kh += nh;
+          uh += nh > 0 ? 1u : 0u;
+        }
+        if (!ok) {
+          // wait until every MMA this thread issued has finished
+          commit(&sh.drain[h]);
+          mbar_drain(&sh.drain[h], 0);
+        }
+      }
+    } else {
+      // ================= Q loader, warp 3 =================
+      const int tl = lane;
+      uint32_t ul[2] = {0, 0};
       bool ok = true;
       for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
         const Tile T = get_tile<MODE>(a, t);
         if (T.skip) continue;
-        for (int j = 0; j < T.n_kv; ++j, ++g) {
-          const uint32_t st = g % NS, u = g / NS;
-          const int z = (int)(T.start + T.kv0 + j * TN);
-          if (u > 0 && !(ok = mbar_wait(&sh.k_empty[st], (u - 1) & 1, abort, status))) break;
-          mbar_expect_tx(&sh.k_full[st], kTile);
-          tma_load_3d(sK + st * kTile, &tmk, &sh.k_full[st], 0, T.g, z);
-          tma_load_3d(sK + st * kTile + kHalf, &tmk, &sh.k_full[st], 64, T.g, z);
-          nk = g + 1;
-          if (u > 0 && !(ok = mbar_wait(&sh.v_empty[st], (u - 1) & 1, abort, status))) break;
-          mbar_expect_tx(&sh.v_full[st], kTile);
-          tma_load_3d(sV + st * kTile, &tmv, &sh.v_full[st], 0, T.g, z);
-          tma_load_3d(sV + st * kTile + kHalf, &tmv, &sh.v_full[st], 64, T.g, z);
-          nv = g + 1;
-        }
-      }
-      if (!ok || *abort) {
-        // let the copies already issued land before the CTA exits
-        for (uint32_t x = nk > NS ? nk - NS : 0; x < nk; ++x)
-          mbar_drain(&sh.k_full[x % NS], (x / NS) & 1);
-        for (uint32_t x = nv > NS ? nv - NS : 0; x < nv; ++x)
-          mbar_drain(&sh.v_full[x % NS], (x / NS) & 1);
-      }
-    }
-  } else if (warp == 1) {
-    // ================= MMA issuer =================
-    if (lane == 0) {
-      const uint32_t tS0 = tmem, tO0 = tmem + 256;
-      uint32_t g = 0, i = 0;
-      bool ok = true, pend = false, plast = false;
-      uint32_t pg = 0, pi = 0;
-      int pj = 0;
-      auto issue_pv = [&](uint32_t gg, uint32_t ii, int jj, bool last) -> bool {
-        const uint32_t ob = ii & 1, bb = gg & 1, st = gg % NS;
-        if (jj == 0 && ii >= 2 && !mbar_wait(&sh.o_free[ob], ((ii >> 1) - 1) & 1, abort, status))
-          return false;
-        if (!mbar_wait(&sh.p_full[bb], (gg >> 1) & 1, abort, status)) return false;
-        if (!mbar_wait(&sh.v_full[st], (gg / NS) & 1, abort, status)) return false;
-        fence_after_sync();
-#pragma unroll
-        for (int kk = 0; kk < TN / 16; ++kk) {
-          const uint64_t bd = desc_sw128(sV + st * kTile + kk * 16 * 128, kHalf, 1024);
-          mma_ts(tO0 + ob * 128, tS0 + bb * 128 + kk * 8, bd, kIdescPV,
-                 (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        commit(&sh.v_empty[st]);
-        commit(&sh.s_free[bb]);
-        if (last) commit(&sh.o_full[ob]);
-        return true;
-      };
-      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-        const Tile T = get_tile<MODE>(a, t);
-        if (T.skip) continue;
-        const uint32_t qb = i & 1;
-        if (!(ok = mbar_wait(&sh.q_full[qb], (i >> 1) & 1, abort, status))) break;
-        for (int j = 0; j < T.n_kv; ++j, ++g) {
-          const uint32_t st = g % NS, bb = g & 1;
-          if (!(ok = mbar_wait(&sh.k_full[st], (g / NS) & 1, abort, status))) break;
-          if (g >= 2 && !(ok = mbar_wait(&sh.s_free[bb], ((g - 2) >> 1) & 1, abort, status)))
-            break;
-          fence_after_sync();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            const uint64_t ad = desc_sw128(sQ + qb * kTile + off, 16, 1024);
-            const uint64_t bd = desc_sw128(sK + st * kTile + off, 16, 1024);
-            mma_ss(tS0 + bb * 128, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
+        for (int h = 0; h < 2; ++h) {
+          if (T.n[h] == 0) continue;
+          if (ul[h] > 0) {
+            ok = mbar_wait(&sh.q_empty[h], (ul[h] - 1) & 1, abort, status);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           }
-          commit(&sh.s_full[bb]);
-          commit(&sh.k_empty[st]);
-          if (j == T.n_kv - 1) commit(&sh.q_empty[qb]);
-          if (pend && !(ok = issue_pv(pg, pi, pj, plast))) break;
-          pend = true;
-          pg = g;
-          pi = i;
-          pj = j;
-          plast = j == T.n_kv - 1;
+          const Tile U = half_view<MODE>(T, h);
+  #pragma unroll
+          for (int hr = 0; hr < TM / kLoaderThreads; ++hr) {
+            const int rr = tl + hr * kLoaderThreads;
+            int64_t qrow = 0;
+            const bool has = q_row_of<MODE>(a, U, rr, qrow);
+            const __nv_bfloat16* src = a.q + (has ? qrow : 0) * (int64_t)D;
+  #pragma unroll
+            for (int c16 = 0; c16 < 16; ++c16) {
+              const uint32_t dst = sQ + h * kTile + (c16 >> 3) * kHalf + rr * 128 +
+                                   ((((uint32_t)c16 & 7u) ^ ((uint32_t)rr & 7u)) << 4);
+              cp_async16(dst, src + c16 * 8, has ? 16u : 0u);
+            }
+          }
+          cp_async_wait_all();
+          fence_proxy_async_smem();
+          mbar_arrive(&sh.q_full[h]);
+          ++ul[h];
         }
-        ++i;
-      }
-      if (ok && pend) ok = issue_pv(pg, pi, pj, plast);
-      if (!ok) {
-        // wait until every MMA issued so far has finished
-        commit(&sh.drain);
-        mbar_drain(&sh.drain, 0);
       }
     }
-  } else if (warp < 6) {
-    // ================= softmax + epilogue, warps 2..5 =================
+  } else {
+    regs_inc();
+    // ====== softmax + epilogue: warps 4..7 half 0, warps 8..11 half 1 ======
+    const int hh = (warp - 4) >> 2;
     const int quarter = warp & 3;          // TMEM lanes this warp may access
     const int r = quarter * 32 + lane;     // query row of this thread
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + hh * 128 + lane_addr;
+    const uint32_t tO = tmem + kOCol + hh * 128 + lane_addr;
     const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;  // softmax scale, base 2
-    uint32_t g = 0, i = 0;
+    const uint32_t stage = sbase + kStageOff + (warp - 4) * 32 * kStageRow;
+    uint32_t kc = 0, uc = 0;
+    int base[2] = {0, 0};  // KV tiles each half processed in earlier units
+    volatile int* exp_cnt = sh.exp_cnt;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-      const Tile T = get_tile<MODE>(a, t);
-      if (T.skip) continue;
+      const Tile T0 = get_tile<MODE>(a, t);
+      if (T0.skip) continue;
+      const int b0 = base[0], b1 = base[1];
+      base[0] += T0.n[0];
+      base[1] += T0.n[1];
+      if (T0.n[hh] == 0) continue;
+      const Tile T = half_view<MODE>(T0, hh);
       const Row R = get_row<MODE>(a, T, r);
-      const uint32_t ob = i & 1;
-      const uint32_t tO = tmem + 256 + ob * 128 + lane_addr;
       float m_i = -INFINITY, l_i = 0.f;
-      for (int j = 0; j < T.n_kv; ++j, ++g) {
-        const uint32_t bb = g & 1;
-        ok = mbar_wait(&sh.s_full[bb], (g >> 1) & 1, abort, status);
+      for (int j = 0; j < T.n_kv; ++j, ++kc) {
+        ok = mbar_wait(&sh.s_full[hh], kc & 1, abort, status);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         fence_after_sync();
-        const uint32_t tS = tmem + bb * 128 + lane_addr;
         float s[TN];
         {
           // issue all four loads, then one wait
@@ -396,7 +489,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           }
         }
         // causal mask on the diagonal tile (CUR / DENSE): key > query
-        if (MODE != HIST && j == T.n_kv - 1) {
+        if (MODE != HIST && T.kv0 + j * TN + TN - 1 > T.p0) {
           const int lim = R.p - (T.kv0 + j * TN);  // last visible column
 #pragma unroll
           for (int x = 0; x < TN; ++x)
@@ -416,12 +509,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
         const bool need = mt > m_i + kRescaleLog2;
         const float m_new = need ? mt : m_i;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
-          // O holds PV of this tile's earlier KV tiles: wait for the last, rescale
-          ok = mbar_wait(&sh.s_free[(g - 1) & 1], ((g - 1) >> 1) & 1, abort, status);
-          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-          fence_after_sync();
+          // O[h] holds PV of the earlier KV tiles: S(j) was committed after
+          // the last of them, so it is complete. Rescale it in place.
           const float alpha = need ? ex2(m_i - m_new) : 1.f;
-#pragma unroll
+#pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t rr[32];
             tmem_ld32(tO + c * 32, rr);
@@ -435,6 +526,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
         if (need) {
           l_i *= ex2(m_i - m_new);
           m_i = m_new;
+        }
+        // CUR / DENSE: the two halves take turns on the exponential unit:
+        // half 1 exponentiates KV tile j after half 0 has, half 0 tile j
+        // after half 1 has done tile j - 1. In anti-phase, one half's PV and
+        // next QK^T run while the other half exponentiates. (HIST units are
+        // only B / 128 KV tiles long and run faster without the turns: one
+        // warp per SM sub-partition reaches only about half the exponential
+        // rate of two.)
+        // Counts only grow, so a half that runs ahead into its next unit
+        // cannot be mistaken for the turn being waited for.
+        if (MODE != HIST && (hh == 0 ? (j >= 1 && j - 1 < T0.n[1]) : (j < T0.n[0]))) {
+          const int need_cnt = 4 * (hh == 0 ? b1 + j : b0 + j + 1);
+          const long long t0 = clock64();
+          while (exp_cnt[hh ^ 1] < need_cnt) {
+            if (*abort) { ok = false; break; }
+            if (clock64() - t0 > kWaitLimitCycles) {
+              *abort = 1;
+              set_status(status, kStTimeout);
+              ok = false;
+              break;
+            }
+          }
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         }
         // P = exp2(s * scale - m) in bf16, two per column, into the S buffer;
         // the row sum is kept in 8 independent partial sums
@@ -454,30 +568,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           }
           tmem_st32(tS + c * 32, pk);
         }
+        __syncwarp();
+        if (lane == 0) atomicAdd(const_cast<int*>(&exp_cnt[hh]), 1);
         tmem_wait_st();
-        const float rowsum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-        l_i += rowsum;
+        l_i += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
         fence_before_sync();
-        mbar_arrive(&sh.p_full[bb]);
+        mbar_arrive(&sh.p_full[hh]);
       }
       if (!ok) break;
-      // ---- epilogue: wait for the tile's last PV, normalise, write
-      ok = mbar_wait(&sh.o_full[ob], (i >> 1) & 1, abort, status);
+      // ---- epilogue: wait for the half's last PV, normalise, write
+      ok = mbar_wait(&sh.o_full[hh], uc & 1, abort, status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       fence_after_sync();
       const float inv_l = 1.f / l_i;
       const float lse = (m_i + log2f(l_i)) * 0.6931471805599453f;
-      // Rows go out through a per-warp staging area so that every global
-      // store instruction writes whole 128-byte segments of 4 or 8 rows.
-      const uint32_t stage = sbase + kStageOff + (warp - 2) * 32 * kStageRow;
       if (MODE == CUR) {
         // Own block done: merge with this row's history partials right here
         // (eq. 7-8 written with lse: w_j = exp(lse_j - m), o = sum_j w_j o_j /
         // sum_j w_j) and write the output; the own result never leaves the
         // SM. Slots 0..slot-1 of the row hold the history partials. Each
         // thread merges its own row with 32 independent 16-byte loads per
-        // slot in flight; the bf16 row then leaves through the staging area
-        // in whole 64-byte pieces.
+        // slot in flight.
         const int slot = R.valid ? (int)(R.prow % dm.topk) : 0;
         const int64_t prow0 = R.valid ? R.prow - slot : 0;
         const int64_t orow = R.valid ? R.t * dm.Hq + R.h : -1;
@@ -490,6 +601,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
 #pragma unroll
           for (int x = 0; x < 32; ++x) o[c * 32 + x] = __uint_as_float(rr[x]) * inv_l;
         }
+        // O[h] is in registers: the next unit's PV may overwrite it
+        fence_before_sync();
+        mbar_arrive(&sh.o_free[hh]);
         if (R.valid) {
           float m = lse;
           for (int j = 0; j < slot; ++j) m = fmaxf(m, a.part_lse[prow0 + j]);
@@ -515,12 +629,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           for (int x = 0; x < D; ++x) o[x] *= inv;
           if (a.lse_out) a.lse_out[orow] = m + logf(L);
         }
+        // the bf16 row leaves through the staging area in 64-byte pieces
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
 #pragma unroll
           for (int x = 0; x < 4; ++x)
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                             stage + lane * 80 + x * 16),
+                             stage + lane * kStageRow + x * 16),
                          "r"(pack_bf16x2(o[c * 32 + 8 * x], o[c * 32 + 8 * x + 1])),
                          "r"(pack_bf16x2(o[c * 32 + 8 * x + 2], o[c * 32 + 8 * x + 3])),
                          "r"(pack_bf16x2(o[c * 32 + 8 * x + 4], o[c * 32 + 8 * x + 5])),
@@ -535,7 +650,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
             uint4 val;
             asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                         : "r"(stage + row * 80 + seg * 16)
+                         : "r"(stage + row * kStageRow + seg * 16)
                          : "memory");
             if (orr >= 0)
               *reinterpret_cast<uint4*>(a.out + orr * D + c * 32 + seg * 8) = val;
@@ -543,12 +658,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           __syncwarp();
         }
       } else {
+        // Rows go out through a per-warp staging area so that every global
+        // store instruction writes whole 64-byte row pieces of 8 rows.
         const int64_t orow = R.valid ? (MODE == DENSE ? R.t * dm.Hq + R.h : R.prow) : -1;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t rr[32];
           tmem_ld32(tO + c * 32, rr);
           tmem_wait_ld();
+          if (c == D / 32 - 1) {
+            // O[h] is in registers: the next unit's PV may overwrite it
+            fence_before_sync();
+            mbar_arrive(&sh.o_free[hh]);
+          }
           if (MODE == DENSE) {
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
@@ -561,12 +683,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
               const uint32_t w3 = pack_bf16x2(__uint_as_float(rr[8 * x + 6]) * inv_l,
                                               __uint_as_float(rr[8 * x + 7]) * inv_l);
               asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                               stage + lane * 80 + x * 16),
+                               stage + lane * kStageRow + x * 16),
                            "r"(w0), "r"(w1), "r"(w2), "r"(w3)
                            : "memory");
             }
             __syncwarp();
-            // 64 bytes per row chunk: 4 lanes per row, 8 rows per instruction
 #pragma unroll
             for (int it = 0; it < 4; ++it) {
               const int row = it * 8 + (lane >> 2), seg = lane & 3;
@@ -574,37 +695,40 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
               uint4 val;
               asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                            : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                           : "r"(stage + row * 80 + seg * 16)
+                           : "r"(stage + row * kStageRow + seg * 16)
                            : "memory");
               if (o >= 0)
                 *reinterpret_cast<uint4*>(a.out + o * D + c * 32 + seg * 8) = val;
             }
+            __syncwarp();
           } else {
 #pragma unroll
-            for (int x = 0; x < 8; ++x)
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                               stage + lane * kStageRow + x * 16),
-                           "r"(__float_as_uint(__uint_as_float(rr[4 * x]) * inv_l)),
-                           "r"(__float_as_uint(__uint_as_float(rr[4 * x + 1]) * inv_l)),
-                           "r"(__float_as_uint(__uint_as_float(rr[4 * x + 2]) * inv_l)),
-                           "r"(__float_as_uint(__uint_as_float(rr[4 * x + 3]) * inv_l))
-                           : "memory");
-            __syncwarp();
-            // 128 bytes per row chunk: 8 lanes per row, 4 rows per instruction
+            for (int sub = 0; sub < 2; ++sub) {  // 16 fp32 columns = 64 bytes per row
 #pragma unroll
-            for (int it = 0; it < 8; ++it) {
-              const int row = it * 4 + (lane >> 3), seg = lane & 7;
-              const int64_t o = __shfl_sync(0xffffffffu, orow, row);
-              uint4 val;
-              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                           : "r"(stage + row * kStageRow + seg * 16)
-                           : "memory");
-              if (o >= 0)
-                *reinterpret_cast<uint4*>(a.part_o + o * D + c * 32 + seg * 4) = val;
+              for (int x = 0; x < 4; ++x)
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                                 stage + lane * kStageRow + x * 16),
+                             "r"(__float_as_uint(__uint_as_float(rr[sub * 16 + 4 * x]) * inv_l)),
+                             "r"(__float_as_uint(__uint_as_float(rr[sub * 16 + 4 * x + 1]) * inv_l)),
+                             "r"(__float_as_uint(__uint_as_float(rr[sub * 16 + 4 * x + 2]) * inv_l)),
+                             "r"(__float_as_uint(__uint_as_float(rr[sub * 16 + 4 * x + 3]) * inv_l))
+                             : "memory");
+              __syncwarp();
+#pragma unroll
+              for (int it = 0; it < 4; ++it) {
+                const int row = it * 8 + (lane >> 2), seg = lane & 3;
+                const int64_t o = __shfl_sync(0xffffffffu, orow, row);
+                uint4 val;
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                             : "r"(stage + row * kStageRow + seg * 16)
+                             : "memory");
+                if (o >= 0)
+                  *reinterpret_cast<uint4*>(a.part_o + o * D + c * 32 + sub * 16 + seg * 4) = val;
+              }
+              __syncwarp();
             }
           }
-          __syncwarp();
         }
         if (R.valid) {
           if (MODE == DENSE) {
@@ -614,40 +738,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           }
         }
       }
-      fence_before_sync();
-      mbar_arrive(&sh.o_free[ob]);
-      ++i;
-    }
-  } else {
-    // ================= Q loaders, warps 6..7 =================
-    const int tl = threadIdx.x - (kThreads - kLoaderThreads);
-    uint32_t i = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-      const Tile T = get_tile<MODE>(a, t);
-      if (T.skip) continue;
-      const uint32_t qb = i & 1;
-      if (i >= 2) {
-        ok = mbar_wait(&sh.q_empty[qb], ((i >> 1) - 1) & 1, abort, status);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      }
-#pragma unroll
-      for (int half_rows = 0; half_rows < TM / kLoaderThreads; ++half_rows) {
-        const int rr = tl + half_rows * kLoaderThreads;
-        int64_t qrow = 0;
-        const bool has = q_row_of<MODE>(a, T, rr, qrow);
-        const __nv_bfloat16* src = a.q + (has ? qrow : 0) * (int64_t)D;
-#pragma unroll
-        for (int c16 = 0; c16 < 16; ++c16) {
-          const uint32_t dst = sQ + qb * kTile + (c16 >> 3) * kHalf + rr * 128 +
-                               ((((uint32_t)c16 & 7u) ^ ((uint32_t)rr & 7u)) << 4);
-          cp_async16(dst, src + c16 * 8, has ? 16u : 0u);
-        }
-      }
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      mbar_arrive(&sh.q_full[qb]);
-      ++i;
+      ++uc;
     }
   }
 
@@ -706,6 +797,11 @@ cudaError_t launch(int64_t tiles, const Args& args, const void* k, const void* v
   if ((e = cudaFuncSetAttribute(attn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 kSmemBytes)))
     return e;
+  // setmaxnreg moves registers between the warp groups inside the block's
+  // launch allocation; never launch with less than the split needs
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, attn_tc_kernel<MODE>))) return e;
+  if (fa.numRegs * kThreads < 128 * kRegsOther + 256 * kRegsSoftmax) return cudaErrorInvalidConfiguration;
   const int64_t grid = tiles < sm_count() ? tiles : sm_count();
   attn_tc_kernel<MODE><<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mk, mv, args);
   return cudaGetLastError();
@@ -722,6 +818,9 @@ Args base_args(const Dims& dm, const Chunk& ch, const void* q, const int32_t* cu
 }
 
 }  // namespace
+
+// Rows of one HIST work unit in the tile table: two query halves.
+int tc_tile_m() { return 2 * TM; }
 
 cudaError_t launch_history_tc(const Dims& dm, const Chunk& ch, const void* q, const void* k,
                               const void* v, const int32_t* cu, const Regroup& rg,
@@ -747,7 +846,7 @@ cudaError_t launch_current_tc(const Dims& dm, const Chunk& ch, const void* q, co
   a.part_lse = pt.lse;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.lse_out = lse;
-  const int64_t tiles = (int64_t)(dm.B / TM) * dm.nb * dm.batch * ch.nq;
+  const int64_t tiles = (int64_t)((dm.B / TM + 1) / 2) * dm.nb * dm.batch * ch.nq;
   a.n_tiles = (int)tiles;
   return launch<CUR>(tiles, a, k, v, st);
 }
@@ -760,7 +859,7 @@ cudaError_t launch_dense_tc(const Dims& dm, const void* q, const void* k, const 
   Args a = base_args(dm, ch, q, cu, status);
   a.out = static_cast<__nv_bfloat16*>(out);
   a.lse_out = lse;
-  const int64_t tiles = (int64_t)((dm.max_seqlen + TM - 1) / TM) * dm.batch * dm.Hq;
+  const int64_t tiles = (int64_t)(((dm.max_seqlen + TM - 1) / TM + 1) / 2) * dm.batch * dm.Hq;
   a.n_tiles = (int)tiles;
   return launch<DENSE>(tiles, a, k, v, st);
 }
