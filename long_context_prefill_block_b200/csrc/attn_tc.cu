@@ -43,6 +43,8 @@
 // kStTimeout, drains the copies and MMAs it issued, frees its TMEM and exits.
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "tc_ptx.cuh"
 
 namespace moba {
@@ -751,57 +753,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
 }
 
 // ---- host side -----------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// [T][H][128] bf16 viewed as (x = d, y = head, z = token); box 64 x 1 x 128.
-cudaError_t make_map(CUtensorMap* map, const void* base, int T, int H) {
-  auto fn = encode_fn();
-  if (!fn) return cudaErrorNotSupported;
-  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
-  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-  const cuuint32_t box[3] = {64, 1, (cuuint32_t)TN};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
-  return n > 0 ? n : 148;
-}
-
 template <int MODE>
 cudaError_t launch(int64_t tiles, const Args& args, const void* k, const void* v,
                    cudaStream_t st) {
   if (tiles <= 0) return cudaSuccess;
   CUtensorMap mk, mv;
   cudaError_t e;
-  if ((e = make_map(&mk, k, args.dm.T, args.dm.Hkv))) return e;
-  if ((e = make_map(&mv, v, args.dm.T, args.dm.Hkv))) return e;
-  if ((e = cudaFuncSetAttribute(attn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                kSmemBytes)))
-    return e;
-  // setmaxnreg moves registers between the warp groups inside the block's
-  // launch allocation; never launch with less than the split needs
-  cudaFuncAttributes fa;
-  if ((e = cudaFuncGetAttributes(&fa, attn_tc_kernel<MODE>))) return e;
-  if (fa.numRegs * kThreads < 128 * kRegsOther + 256 * kRegsSoftmax) return cudaErrorInvalidConfiguration;
+  if ((e = make_head_map(&mk, k, args.dm.T, args.dm.Hkv, TN))) return e;
+  if ((e = make_head_map(&mv, v, args.dm.T, args.dm.Hkv, TN))) return e;
+  // Once per device: allow the shared memory, and check that the launch
+  // allocates the registers the setmaxnreg split needs (setmaxnreg moves
+  // registers between the warp groups inside the block's allocation).
+  static std::mutex mu;
+  static int ready[kMaxDevices] = {};  // 0 unknown, 1 ready, -1 unusable
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev))) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (ready[dev] == 0) {
+      if ((e = cudaFuncSetAttribute(attn_tc_kernel<MODE>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes)))
+        return e;
+      cudaFuncAttributes fa;
+      if ((e = cudaFuncGetAttributes(&fa, attn_tc_kernel<MODE>))) return e;
+      ready[dev] = fa.numRegs * kThreads >= 128 * kRegsOther + 256 * kRegsSoftmax ? 1 : -1;
+    }
+  }
+  if (ready[dev] < 0) return cudaErrorInvalidConfiguration;
   const int64_t grid = tiles < sm_count() ? tiles : sm_count();
   attn_tc_kernel<MODE><<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mk, mv, args);
   return cudaGetLastError();

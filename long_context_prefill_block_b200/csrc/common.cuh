@@ -100,6 +100,10 @@ namespace moba {
 
 cudaError_t launch_meanpool(const Dims& dm, const void* k, const int32_t* cu, float* kbar,
                             int* status, cudaStream_t st);
+// Tensor-core gate (bf16, d = 128, at most 256 blocks per sequence).
+bool gate_tc_supported(const Dims& dm);
+cudaError_t launch_gate_tc(const Dims& dm, const void* q, const float* kbar, const int32_t* cu,
+                           int32_t* idx, int* status, cudaStream_t st);
 cudaError_t launch_gate(const Dims& dm, const void* q, const float* kbar, const int32_t* cu,
                         int32_t* idx, int* status, cudaStream_t st);
 

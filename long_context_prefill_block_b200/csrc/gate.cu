@@ -221,6 +221,7 @@ cudaError_t by_k(const Dims& dm, const void* q, const float* kbar, const int32_t
 cudaError_t launch_gate(const Dims& dm, const void* q, const float* kbar, const int32_t* cu,
                         int32_t* idx, int* status, cudaStream_t st) {
   if (dm.batch == 0 || dm.max_seqlen == 0) return cudaSuccess;
+  if (gate_tc_supported(dm)) return launch_gate_tc(dm, q, kbar, cu, idx, status, st);
   if (dm.dtype == kBF16)
     return dm.d == 128 ? by_k<__nv_bfloat16, 128>(dm, q, kbar, cu, idx, status, st)
                        : by_k<__nv_bfloat16, 64>(dm, q, kbar, cu, idx, status, st);
