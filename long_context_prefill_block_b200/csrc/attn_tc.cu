@@ -76,6 +76,7 @@ constexpr uint32_t kQOff = 0;          // Q[2], one per query half
 constexpr uint32_t kKOff = 2 * kTile;  // K[NS]
 constexpr uint32_t kVOff = kKOff + NS * kTile;
 constexpr uint32_t kStageRow = 80;     // bytes per staged row chunk: 64 + 16 pad
+constexpr uint32_t kStageRow128 = 144; // 128-byte row pieces, 16 rows at a time (fits 32 x 80)
 constexpr uint32_t kStageOff = kVOff + NS * kTile;  // epilogue staging, 32 rows per softmax warp
 constexpr uint32_t kStageBytes = 8 * 32 * kStageRow;
 constexpr uint32_t kSmemBytes = kStageOff + kStageBytes + 1024;  // + 1024-byte alignment slack
@@ -616,14 +617,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           for (int j = 0; j < slot; ++j) {
             const float wj = ex2((a.part_lse[prow0 + j] - m) * 1.4426950408889634f);
             L += wj;
-            const float4* src = reinterpret_cast<const float4*>(a.part_o + (prow0 + j) * D);
+            // 32-byte loads: half the load instructions (each touches one
+            // line per row of the warp) of 16-byte ones
+            const float* src = a.part_o + (prow0 + j) * D;
 #pragma unroll
-            for (int x4 = 0; x4 < D / 4; ++x4) {
-              const float4 v = src[x4];
-              o[4 * x4] = fmaf(wj, v.x, o[4 * x4]);
-              o[4 * x4 + 1] = fmaf(wj, v.y, o[4 * x4 + 1]);
-              o[4 * x4 + 2] = fmaf(wj, v.z, o[4 * x4 + 2]);
-              o[4 * x4 + 3] = fmaf(wj, v.w, o[4 * x4 + 3]);
+            for (int x8 = 0; x8 < D / 8; ++x8) {
+              float v[8];
+              ld_global_v8(src + 8 * x8, v);
+#pragma unroll
+              for (int u = 0; u < 8; ++u) o[8 * x8 + u] = fmaf(wj, v[u], o[8 * x8 + u]);
             }
           }
           const float inv = 1.f / L;
@@ -705,28 +707,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
             __syncwarp();
           } else {
 #pragma unroll
-            for (int sub = 0; sub < 2; ++sub) {  // 16 fp32 columns = 64 bytes per row
+            for (int rd = 0; rd < 2; ++rd) {  // 32 fp32 columns = 128 bytes per row, 16 rows at a time
+              if ((lane >> 4) == rd) {
 #pragma unroll
-              for (int x = 0; x < 4; ++x)
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                                 stage + lane * kStageRow + x * 16),
-                             "r"(__float_as_uint(__uint_as_float(rr[sub * 16 + 4 * x]) * inv_l)),
-                             "r"(__float_as_uint(__uint_as_float(rr[sub * 16 + 4 * x + 1]) * inv_l)),
-                             "r"(__float_as_uint(__uint_as_float(rr[sub * 16 + 4 * x + 2]) * inv_l)),
-                             "r"(__float_as_uint(__uint_as_float(rr[sub * 16 + 4 * x + 3]) * inv_l))
-                             : "memory");
+                for (int x = 0; x < 8; ++x)
+                  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                                   stage + (lane & 15) * kStageRow128 + x * 16),
+                               "r"(__float_as_uint(__uint_as_float(rr[4 * x]) * inv_l)),
+                               "r"(__float_as_uint(__uint_as_float(rr[4 * x + 1]) * inv_l)),
+                               "r"(__float_as_uint(__uint_as_float(rr[4 * x + 2]) * inv_l)),
+                               "r"(__float_as_uint(__uint_as_float(rr[4 * x + 3]) * inv_l))
+                               : "memory");
+              }
               __syncwarp();
+              // 8 lanes per row, 4 rows per instruction
 #pragma unroll
               for (int it = 0; it < 4; ++it) {
-                const int row = it * 8 + (lane >> 2), seg = lane & 3;
-                const int64_t o = __shfl_sync(0xffffffffu, orow, row);
+                const int row = it * 4 + (lane >> 3), seg = lane & 7;
+                const int64_t o = __shfl_sync(0xffffffffu, orow, rd * 16 + row);
                 uint4 val;
                 asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                              : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                             : "r"(stage + row * kStageRow + seg * 16)
+                             : "r"(stage + row * kStageRow128 + seg * 16)
                              : "memory");
                 if (o >= 0)
-                  *reinterpret_cast<uint4*>(a.part_o + o * D + c * 32 + sub * 16 + seg * 4) = val;
+                  *reinterpret_cast<uint4*>(a.part_o + o * D + c * 32 + seg * 4) = val;
               }
               __syncwarp();
             }
