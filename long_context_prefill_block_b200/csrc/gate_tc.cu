@@ -30,8 +30,8 @@ constexpr int kThreads = 256;                // row r: threads r and r + 128
 constexpr int kTileRows = 128;               // queries per tile
 constexpr uint32_t kQHalf = 128 * 128;       // one 64-column half of a Q tile
 constexpr uint32_t kQTile = 2 * kQHalf;
-constexpr int kMaxBlocks = 128;              // beyond this the SIMT gate's 4-way split scan is faster
-constexpr int kCuSmem = 1025;                // sequence offsets kept in shared memory
+constexpr int kMaxBlocks = 256;              // MMA N limit
+constexpr int kCuSmem = 257;                 // sequence offsets kept in shared memory (batch <= 256)
 
 struct GateArgs {
   Dims dm;
@@ -288,14 +288,30 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmq, const GateArgs a) {
     const int cw = __reduce_max_sync(0xffffffffu, c);  // columns this warp needs
     const uint32_t taddr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     for (int cb = part; cb * 32 < cw; cb += 2) {
-      uint32_t rr[32];
-      tmem_ld32(taddr + cb * 32, rr);
-      tmem_wait_ld();
+      if (KM <= 4) {
+        uint32_t rr[32];
+        tmem_ld32(taddr + cb * 32, rr);
+        tmem_wait_ld();
 #pragma unroll
-      for (int xx = 0; xx < 32; ++xx) {
-        const int i = cb * 32 + xx;
-        if (cb * 32 + xx >= cw) break;  // past every row's candidates in this warp
-        if (i < c) insert_scan<KM>(ts, ti, __uint_as_float(rr[xx]), i);
+        for (int xx = 0; xx < 32; ++xx) {
+          const int i = cb * 32 + xx;
+          if (cb * 32 + xx >= cw) break;  // past every row's candidates in this warp
+          if (i < c) insert_scan<KM>(ts, ti, __uint_as_float(rr[xx]), i);
+        }
+      } else {
+        // long lists: four columns per step, so the unrolled insertion code
+        // stays small enough for the instruction cache
+#pragma unroll 1
+        for (int x4 = 0; x4 < 8 && cb * 32 + x4 * 4 < cw; ++x4) {
+          uint32_t rr[4];
+          tmem_ld4(taddr + cb * 32 + x4 * 4, rr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = cb * 32 + x4 * 4 + u;
+            if (i < c) insert_scan<KM>(ts, ti, __uint_as_float(rr[u]), i);
+          }
+        }
       }
     }
     // the second thread's list goes through TMEM (same lane, spare columns)
