@@ -71,6 +71,12 @@ typedef struct {
   int block_size;    /* B >= 1 */
   int topk;          /* k, 1 <= k <= 32; the current block uses one slot */
   moba_dtype dtype;
+  int routing;       /* 0 (default): every query head chooses its own blocks.
+                        1: the query heads of a kv head's group share one choice,
+                        made on the group's mean score (1/grp) sum_h q_h . kbar_i
+                        (PaperTrace "2.1.3 MoBA", section 5.4, multi-head
+                        settings: a group sharing candidates must aggregate its
+                        heads' scores; the mean is this library's reading). */
 } moba_params;
 
 /* Number of key blocks reserved per sequence: ceil(max_seqlen / B). */

@@ -32,7 +32,8 @@ class MobaParams(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int), ("total_tokens", ctypes.c_int),
                 ("max_seqlen", ctypes.c_int), ("num_q_heads", ctypes.c_int),
                 ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
-                ("block_size", ctypes.c_int), ("topk", ctypes.c_int), ("dtype", ctypes.c_int)]
+                ("block_size", ctypes.c_int), ("topk", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("routing", ctypes.c_int)]
 
 
 class MobaError(RuntimeError):
@@ -78,7 +79,8 @@ def _check(fn: str, code: int) -> None:
 
 
 def make_params(q: torch.Tensor, k: torch.Tensor, cu_seqlens: torch.Tensor, block_size: int,
-                topk: int, max_seqlen: Optional[int] = None) -> MobaParams:
+                topk: int, max_seqlen: Optional[int] = None,
+                shared_routing: bool = False) -> MobaParams:
     T, Hq, d = q.shape
     Hkv = k.shape[1]
     batch = cu_seqlens.numel() - 1
@@ -91,7 +93,8 @@ def make_params(q: torch.Tensor, k: torch.Tensor, cu_seqlens: torch.Tensor, bloc
         dt = MOBA_F32
     else:
         raise TypeError(f"unsupported dtype {q.dtype}")
-    return MobaParams(batch, T, max_seqlen, Hq, Hkv, d, block_size, topk, dt)
+    return MobaParams(batch, T, max_seqlen, Hq, Hkv, d, block_size, topk, dt,
+                      1 if shared_routing else 0)
 
 
 def _ptr(x: Optional[torch.Tensor]):
@@ -139,10 +142,11 @@ def moba_meanpool(k: torch.Tensor, cu_seqlens: torch.Tensor, block_size: int,
 
 
 def moba_gate_topk(q, k, cu_seqlens, block_size: int, topk: int, max_seqlen=None,
-                   ws: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Chosen blocks per (token, q head): int32 [T, Hq, topk], ascending, -1 padded."""
+                   ws: Optional[torch.Tensor] = None, shared_routing: bool = False) -> torch.Tensor:
+    """Chosen blocks per (token, q head): int32 [T, Hq, topk], ascending, -1 padded.
+    shared_routing: the q heads of a kv head's group share the blocks of their mean score."""
     _check_inputs(q, k)
-    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen)
+    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen, shared_routing)
     cu = _dev_i32(cu_seqlens, q.device)
     ws = workspace(p, q.device) if ws is None else ws
     idx = torch.empty((p.total_tokens, p.num_q_heads, topk), dtype=torch.int32, device=q.device)
@@ -153,7 +157,8 @@ def moba_gate_topk(q, k, cu_seqlens, block_size: int, topk: int, max_seqlen=None
 
 
 def moba_gate_topk_noalloc(q, k, cu_seqlens, block_size: int, topk: int, max_seqlen=None,
-                           idx: Optional[torch.Tensor] = None) -> torch.Tensor:
+                           idx: Optional[torch.Tensor] = None,
+                           shared_routing: bool = False) -> torch.Tensor:
     """moba_gate_topk without a workspace, for callers that cannot allocate
     device memory: the block means use a fixed 4 MiB array inside the
     library (see include/moba.h for the limit and the sharing rules)."""
@@ -162,7 +167,7 @@ def moba_gate_topk_noalloc(q, k, cu_seqlens, block_size: int, topk: int, max_seq
     fn = L.moba_gate_topk_noalloc
     fn.argtypes = [ctypes.POINTER(MobaParams)] + [ctypes.c_void_p] * 5
     fn.restype = ctypes.c_int
-    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen)
+    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen, shared_routing)
     cu = _dev_i32(cu_seqlens, q.device)
     if idx is None:
         idx = torch.empty((p.total_tokens, p.num_q_heads, topk), dtype=torch.int32,
@@ -174,10 +179,11 @@ def moba_gate_topk_noalloc(q, k, cu_seqlens, block_size: int, topk: int, max_seq
 
 def moba_forward(q, k, v, cu_seqlens, block_size: int, topk: int, max_seqlen=None,
                  return_lse: bool = False, ws: Optional[torch.Tensor] = None,
-                 out: Optional[torch.Tensor] = None):
-    """MoBA prefill forward: out [T, Hq, d] (input dtype) and optionally lse [T, Hq]."""
+                 out: Optional[torch.Tensor] = None, shared_routing: bool = False):
+    """MoBA prefill forward: out [T, Hq, d] (input dtype) and optionally lse [T, Hq].
+    shared_routing: the q heads of a kv head's group share the blocks of their mean score."""
     _check_inputs(q, k, v)
-    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen)
+    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen, shared_routing)
     cu = _dev_i32(cu_seqlens, q.device)
     ws = workspace(p, q.device) if ws is None else ws
     out = torch.empty_like(q) if out is None else out

@@ -43,6 +43,7 @@ moba_status validate(const moba_params* p, Dims& dm) {
       p->num_kv_heads <= 0 || p->num_q_heads % p->num_kv_heads != 0 || p->block_size <= 0 ||
       p->topk <= 0)
     return MOBA_ERR_INVALID_ARG;
+  if (p->routing != 0 && p->routing != 1) return MOBA_ERR_INVALID_ARG;
   if (p->dtype != MOBA_BF16 && p->dtype != MOBA_F32) return MOBA_ERR_UNSUPPORTED;
   if (p->head_dim != 64 && p->head_dim != 128) return MOBA_ERR_UNSUPPORTED;
   if (p->topk > 32) return MOBA_ERR_UNSUPPORTED;
@@ -59,6 +60,7 @@ moba_status validate(const moba_params* p, Dims& dm) {
   dm.topk = p->topk;
   dm.nb = (int)(((int64_t)p->max_seqlen + p->block_size - 1) / p->block_size);
   dm.dtype = p->dtype == MOBA_BF16 ? kBF16 : kF32;
+  dm.shared = p->routing;
   return MOBA_OK;
 }
 

@@ -27,6 +27,7 @@ struct Dims {
   int topk;        // k
   int nb;          // blocks reserved per sequence = ceil(max_seqlen / B)
   int dtype;       // kBF16 / kF32
+  int shared;      // 1: a kv head's query heads share the blocks of their mean score
 };
 
 // Work of one pass over a group of kv heads [g0, g0 + ng): its q heads are

@@ -55,8 +55,11 @@ __global__ void __launch_bounds__(kThreads) gate_kernel(Dims dm, const T* __rest
   float(*kb)[D + 4] = reinterpret_cast<float(*)[D + 4]>(gsm + kQ * (D + 4));      // [kCh]
   float(*sc)[kCh + 1] = reinterpret_cast<float(*)[kCh + 1]>(gsm + (kQ + kCh) * (D + 4));
 
-  const int b = blockIdx.y, h = blockIdx.z;
-  const int g = h / (dm.Hq / dm.Hkv);
+  // blockIdx.z: the q head, or with shared routing the kv head, whose group
+  // of nh q heads is scored by the sum of their q rows (the mean's ranking)
+  const int b = blockIdx.y, grp = dm.Hq / dm.Hkv;
+  const int g = dm.shared ? (int)blockIdx.z : (int)blockIdx.z / grp;
+  const int h0 = dm.shared ? g * grp : (int)blockIdx.z, nh = dm.shared ? grp : 1;
   int64_t start;
   int len;
   if (!seq_bounds(dm, cu, b, start, len, status)) return;
@@ -67,11 +70,15 @@ __global__ void __launch_bounds__(kThreads) gate_kernel(Dims dm, const T* __rest
   for (int e = threadIdx.x; e < kQ * TPR; e += kThreads) {
     const int r = e / TPR, l = e % TPR;
     float x[VEC];
-    if (p0 + r < len) {
-      Vec16<T>::load(q + ((start + p0 + r) * dm.Hq + h) * (int64_t)D + l * VEC, x);
-    } else {
 #pragma unroll
-      for (int u = 0; u < VEC; ++u) x[u] = 0.f;
+    for (int u = 0; u < VEC; ++u) x[u] = 0.f;
+    if (p0 + r < len) {
+      for (int hh = 0; hh < nh; ++hh) {
+        float y[VEC];
+        Vec16<T>::load(q + ((start + p0 + r) * dm.Hq + h0 + hh) * (int64_t)D + l * VEC, y);
+#pragma unroll
+        for (int u = 0; u < VEC; ++u) x[u] += y[u];
+      }
     }
 #pragma unroll
     for (int u = 0; u < VEC; ++u) qs[r][l * VEC + u] = x[u];
@@ -184,17 +191,19 @@ __global__ void __launch_bounds__(kThreads) gate_kernel(Dims dm, const T* __rest
       }
     }
   }
-  int32_t* row = idx + ((start + p) * dm.Hq + h) * (int64_t)dm.topk;
+  for (int hh = 0; hh < nh; ++hh) {
+    int32_t* row = idx + ((start + p) * dm.Hq + h0 + hh) * (int64_t)dm.topk;
 #pragma unroll
-  for (int r = 0; r <= KM; ++r) {
-    if (r < dm.topk) row[r] = r < hsel ? sel[r < KM ? r : KM - 1] : (r == hsel ? c : -1);
+    for (int r = 0; r <= KM; ++r) {
+      if (r < dm.topk) row[r] = r < hsel ? sel[r < KM ? r : KM - 1] : (r == hsel ? c : -1);
+    }
   }
 }
 
 template <typename T, int D, int KM>
 cudaError_t run(const Dims& dm, const void* q, const float* kbar, const int32_t* cu, int32_t* idx,
                 int* status, cudaStream_t st) {
-  dim3 grid((dm.max_seqlen + kQ - 1) / kQ, dm.batch, dm.Hq);
+  dim3 grid((dm.max_seqlen + kQ - 1) / kQ, dm.batch, dm.shared ? dm.Hkv : dm.Hq);
   const size_t smem = sizeof(float) * ((kQ + kCh) * (D + 4) + kQ * (kCh + 1));
   cudaError_t e = cudaFuncSetAttribute(gate_kernel<T, D, KM>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

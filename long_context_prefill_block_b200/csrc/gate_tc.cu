@@ -93,10 +93,11 @@ struct Item {
 __device__ __forceinline__ Item decode(const GateArgs& a, const int32_t* cu, int it) {
   const Dims& dm = a.dm;
   const int grp = dm.Hq / dm.Hkv;
+  const int per_tile = dm.shared ? 1 : grp;  // items per (query tile, kv head)
   const int nqt = (dm.max_seqlen + kTileRows - 1) / kTileRows;
   Item x;
-  const int hl = it % grp;
-  int rest = it / grp;
+  const int hl = it % per_tile;
+  int rest = it / per_tile;
   const int qt = rest % nqt;
   rest /= nqt;
   x.g = rest % dm.Hkv;
@@ -171,12 +172,15 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmq, const GateArgs a) {
   volatile int* abort = &abort_flag;
   int* status = a.status;
 
-  auto issue_q = [&](int it, uint32_t buf) {
+  // Q tiles per item: with shared routing every q head of the group, whose
+  // scores accumulate in TMEM (their sum ranks like their mean)
+  const int nh = dm.shared ? dm.Hq / dm.Hkv : 1;
+  auto issue_q = [&](int it, int hh, uint32_t buf) {
     const Item x = decode(a, cu, it);
     mbar_expect_tx(&q_full[buf], kQTile);
     const int z = (int)(x.start + x.p0);
-    tma_load_3d(sQ + buf * kQTile, &tmq, &q_full[buf], 0, x.h, z);
-    tma_load_3d(sQ + buf * kQTile + kQHalf, &tmq, &q_full[buf], 64, x.h, z);
+    tma_load_3d(sQ + buf * kQTile, &tmq, &q_full[buf], 0, x.h + hh, z);
+    tma_load_3d(sQ + buf * kQTile + kQHalf, &tmq, &q_full[buf], 64, x.h + hh, z);
   };
 
   int slot = 0;
@@ -184,7 +188,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmq, const GateArgs a) {
   uint32_t nq = 0, nmma = 0;  // Q tiles requested / consumed so far; MMA groups
   uint32_t n_issued = 0;
   if (it >= 0 && tid == 0) {
-    issue_q(it, 0);
+    issue_q(it, 0, 0);
     n_issued = 1;
   }
   int cur_b = -1, cur_g = -1;
@@ -232,45 +236,51 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmq, const GateArgs a) {
       cur_b = x.b;
       cur_g = x.g;
     }
-    const uint32_t qb = nq % a.qbuf;
-    ok = mbar_wait(&q_full[qb], (nq / a.qbuf) & 1, abort, status);
-    if (!ok) break;
-    ++nq;
     // blocks any row of the tile may choose: i < c(p) <= c_max
     const int c_max = (min(x.p0 + kTileRows, x.len) - 1) / dm.B;
     const int N = ((c_max + 15) / 16) * 16;
-    if (N > 0 && tid == 0) {
-      fence_after_sync();
-      const uint32_t idesc = idesc_bf16(kTileRows, N, false, false);
-#pragma unroll 1
-      for (int t = 0; t < 3; ++t)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ko = (kk >> 2) * kQHalf + (kk & 3) * 32;
-          const uint64_t ad = desc_sw128(sQ + qb * kQTile + ko, 16, 1024);
-          const uint64_t bd =
-              desc_sw128(sK + t * 2 * kTermHalf + (kk >> 2) * kTermHalf + (kk & 3) * 32, 16, 1024);
-          mma_ss(tmem, ad, bd, idesc, (t > 0 || kk > 0) ? 1u : 0u);
-        }
-      commit(&mma_done);
-    }
     int nslot = slot + 1;
     const int nxt = next_valid(a, cu, nslot);
-    if (a.qbuf == 2 && tid == 0 && nxt >= 0) {
-      // the other buffer's last reader (the previous tile's MMA) is done
-      issue_q(nxt, n_issued % 2);
-      ++n_issued;
-    }
-    if (N > 0) {
-      ok = mbar_wait(&mma_done, nmma & 1, abort, status);
-      ++nmma;
+    for (int hh = 0; ok && hh < nh; ++hh) {
+      const uint32_t qb = nq % a.qbuf;
+      ok = mbar_wait(&q_full[qb], (nq / a.qbuf) & 1, abort, status);
       if (!ok) break;
-      fence_after_sync();
+      ++nq;
+      if (N > 0 && tid == 0) {
+        fence_after_sync();
+        const uint32_t idesc = idesc_bf16(kTileRows, N, false, false);
+#pragma unroll 1
+        for (int t = 0; t < 3; ++t)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t ko = (kk >> 2) * kQHalf + (kk & 3) * 32;
+            const uint64_t ad = desc_sw128(sQ + qb * kQTile + ko, 16, 1024);
+            const uint64_t bd = desc_sw128(
+                sK + t * 2 * kTermHalf + (kk >> 2) * kTermHalf + (kk & 3) * 32, 16, 1024);
+            mma_ss(tmem, ad, bd, idesc, (hh > 0 || t > 0 || kk > 0) ? 1u : 0u);
+          }
+        commit(&mma_done);
+      }
+      // the next Q tile: this item's next head, else the next item's first
+      const bool more = hh + 1 < nh;
+      const bool has_next = more || nxt >= 0;
+      if (a.qbuf == 2 && tid == 0 && has_next) {
+        // the other buffer's last reader (the previous tile's MMA) is done
+        issue_q(more ? it : nxt, more ? hh + 1 : 0, n_issued % 2);
+        ++n_issued;
+      }
+      if (N > 0) {
+        ok = mbar_wait(&mma_done, nmma & 1, abort, status);
+        ++nmma;
+        if (!ok) break;
+        fence_after_sync();
+      }
+      if (a.qbuf == 1 && tid == 0 && has_next) {
+        issue_q(more ? it : nxt, more ? hh + 1 : 0, 0);
+        ++n_issued;
+      }
     }
-    if (a.qbuf == 1 && tid == 0 && nxt >= 0) {
-      issue_q(nxt, 0);
-      ++n_issued;
-    }
+    if (!ok) break;
     // ---- selection: row rr of the tile (TMEM lane rr); thread rr scans the
     // even 32-column chunks of the candidates, thread rr + 128 the odd ones,
     // then the first merges the second's list
@@ -362,9 +372,11 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmq, const GateArgs a) {
             sel[j] = sel[j + 1];
             sel[j + 1] = s;
           }
-      int32_t* row = a.idx + ((x.start + p) * dm.Hq + x.h) * (int64_t)dm.topk;
-      for (int r = 0; r < dm.topk; ++r)
-        row[r] = r < hsel ? sel[r < KM ? r : KM - 1] : (r == hsel ? c : -1);
+      for (int hh = 0; hh < nh; ++hh) {
+        int32_t* row = a.idx + ((x.start + p) * dm.Hq + x.h + hh) * (int64_t)dm.topk;
+        for (int r = 0; r < dm.topk; ++r)
+          row[r] = r < hsel ? sel[r < KM ? r : KM - 1] : (r == hsel ? c : -1);
+      }
     }
     // TMEM and this Q buffer are free again
     fence_before_sync();
@@ -447,7 +459,7 @@ cudaError_t launch_gate_tc(const Dims& dm, const void* q, const float* kbar, con
   a.idx = idx;
   a.status = status;
   const int nqt = (dm.max_seqlen + kTileRows - 1) / kTileRows;
-  const int64_t ipg = (int64_t)nqt * (dm.Hq / dm.Hkv);
+  const int64_t ipg = (int64_t)nqt * (dm.shared ? 1 : dm.Hq / dm.Hkv);
   if ((int64_t)dm.batch * dm.Hkv * ipg > INT_MAX) return cudaErrorInvalidValue;
   a.groups = dm.batch * dm.Hkv;
   a.ipg = (int)ipg;

@@ -35,6 +35,10 @@ def _lib():
             "oracle_forward_mask": [P, P, P, I, P, I, I, I, I, I, I, P, P],
             "oracle_forward_two_branch": [P, P, P, I, P, I, I, I, I, I, I, I, P],
             "oracle_dense_causal": [P, P, P, I, P, I, I, I, I, P, P],
+            "oracle_gate_topk_routed": [P, P, I, P, I, I, I, I, I, I, I, P, P],
+            "oracle_forward_routed": [P, P, P, I, P, I, I, I, I, I, I, I, P, P, P, P, P],
+            "oracle_forward_rows_routed": [P, P, P, I, P, I, I, I, I, I, I, I, P, L, P, P, P, P, P,
+                                           P],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -113,22 +117,25 @@ def meanpool(k, cu_seqlens, block_size):
     return out
 
 
-def gate_topk(q, k, cu_seqlens, block_size, topk):
-    """(idx [T, Hq, topk] int32, gap [T, Hq] float64)."""
+def gate_topk(q, k, cu_seqlens, block_size, topk, shared_routing=False):
+    """(idx [T, Hq, topk] int32, gap [T, Hq] float64). shared_routing: every
+    query head of a kv head's group takes the blocks chosen by the group's
+    mean score."""
     qr, kr, _, dt = _qkv(q, k, None)
     cu = _i32(cu_seqlens)
     T, Hq, d = qr.shape
     Hkv = kr.shape[1]
     idx = np.full((T, Hq, topk), -1, dtype=np.int32)
     gap = np.zeros((T, Hq), dtype=np.float64)
-    rc = _lib().oracle_gate_topk(_ptr(qr), _ptr(kr), dt, _ptr(cu), len(cu) - 1, Hq, Hkv, d,
-                                 block_size, topk, _ptr(idx), _ptr(gap))
+    rc = _lib().oracle_gate_topk_routed(_ptr(qr), _ptr(kr), dt, _ptr(cu), len(cu) - 1, Hq, Hkv, d,
+                                        block_size, topk, int(bool(shared_routing)), _ptr(idx),
+                                        _ptr(gap))
     if rc:
         raise ValueError("oracle_gate_topk: invalid arguments")
     return idx, gap
 
 
-def forward(q, k, v, cu_seqlens, block_size, topk, indices=None):
+def forward(q, k, v, cu_seqlens, block_size, topk, indices=None, shared_routing=False):
     """Full forward by definition: (out [T,Hq,d], lse [T,Hq], idx [T,Hq,topk], nkeys [T,Hq])."""
     qr, kr, vr, dt = _qkv(q, k, v)
     cu = _i32(cu_seqlens)
@@ -139,16 +146,16 @@ def forward(q, k, v, cu_seqlens, block_size, topk, indices=None):
     lse = np.zeros((T, Hq), dtype=np.float64)
     idx = np.full((T, Hq, topk), -1, dtype=np.int32)
     nkeys = np.zeros((T, Hq), dtype=np.int64)
-    rc = _lib().oracle_forward(_ptr(qr), _ptr(kr), _ptr(vr), dt, _ptr(cu), len(cu) - 1, Hq, Hkv, d,
-                               block_size, topk, _ptr(idx_in), _ptr(out), _ptr(lse), _ptr(idx),
-                               _ptr(nkeys))
+    rc = _lib().oracle_forward_routed(_ptr(qr), _ptr(kr), _ptr(vr), dt, _ptr(cu), len(cu) - 1, Hq,
+                                      Hkv, d, block_size, topk, int(bool(shared_routing)),
+                                      _ptr(idx_in), _ptr(out), _ptr(lse), _ptr(idx), _ptr(nkeys))
     if rc:
         raise ValueError("oracle_forward: invalid arguments")
     return out, lse, idx, nkeys
 
 
 def forward_rows(q, k, v, cu_seqlens, block_size, topk, rows, indices=None, q_rows=None,
-                 num_q_heads=None):
+                 num_q_heads=None, shared_routing=False):
     """Sampled forward on rows (row = t*Hq + h): (out [n,d], lse [n], idx [n,topk], gap [n]).
 
     With q_rows ([n, d], the q vectors of the listed rows) q may be None and
@@ -175,10 +182,11 @@ def forward_rows(q, k, v, cu_seqlens, block_size, topk, rows, indices=None, q_ro
     lse = np.zeros(n, dtype=np.float64)
     idx = np.full((n, topk), -1, dtype=np.int32)
     gap = np.zeros(n, dtype=np.float64)
-    rc = _lib().oracle_forward_rows(_ptr(qbase), _ptr(kr), _ptr(vr), dt, _ptr(cu), len(cu) - 1,
-                                    Hq, Hkv, d, block_size, topk, _ptr(rows), n, _ptr(idx_in),
-                                    _ptr(out), _ptr(lse), _ptr(idx), _ptr(gap),
-                                    _ptr(qr) if q_rows is not None else None)
+    rc = _lib().oracle_forward_rows_routed(_ptr(qbase), _ptr(kr), _ptr(vr), dt, _ptr(cu),
+                                           len(cu) - 1, Hq, Hkv, d, block_size, topk,
+                                           int(bool(shared_routing)), _ptr(rows), n, _ptr(idx_in),
+                                           _ptr(out), _ptr(lse), _ptr(idx), _ptr(gap),
+                                           _ptr(qr) if q_rows is not None else None)
     if rc:
         raise ValueError("oracle_forward_rows: invalid arguments")
     return out, lse, idx, gap

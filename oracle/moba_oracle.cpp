@@ -33,6 +33,16 @@
 //   oracle_forward_two_branch keeps (m, l, u) for the current-block and the
 //                             history branch and merges them with [PT §2]
 //                             eq. (7)-(8).
+//
+// Routing variant ([PT §5.4], the paragraph on multi-head settings: a group
+// of heads may share its candidate blocks, the routing score then has to
+// aggregate the heads' needs): with shared routing every query head of a kv
+// head's group gets the same blocks, chosen by the group's MEAN score
+//   s_i = (1/grp) sum_{h in group} q_{p,h} . kbar_i
+// under the same causal mask, forced own block and tie rule. (The pages do
+// not fix the aggregate; the mean, which averages the heads' needs, is the
+// reading taken.) The *_routed entry points take routing = 0 (per head, the
+// default everywhere else) or 1 (shared by the group).
 
 #include <algorithm>
 #include <cmath>
@@ -55,6 +65,7 @@ struct Problem {
   int dtype;
   const int32_t* cu;  // [batch + 1]
   int batch, Hq, Hkv, d, B, topk;
+  int shared;  // 1: the kv head's query heads share their blocks (mean score)
 };
 
 // Exact widening of a stored element to double.
@@ -112,11 +123,17 @@ void select_blocks(const Problem& P, int64_t t, int h, int64_t p, const std::vec
   const int64_t c = p / P.B;
   std::vector<std::pair<double, int64_t>> s;
   s.reserve(static_cast<size_t>(c));
+  const int grp = P.Hq / P.Hkv;
+  const int h0 = P.shared ? (h / grp) * grp : h, nh_score = P.shared ? grp : 1;
   for (int64_t i = 0; i < c; ++i) {
-    double acc = 0.0;
     const double* kb = &kbar[static_cast<size_t>(i * P.d)];
-    for (int x = 0; x < P.d; ++x) acc += load(P.q, P.dtype, q_off(P, t, h) + x) * kb[x];
-    s.emplace_back(acc, i);
+    double sum = 0.0;
+    for (int hh = h0; hh < h0 + nh_score; ++hh) {
+      double acc = 0.0;
+      for (int x = 0; x < P.d; ++x) acc += load(P.q, P.dtype, q_off(P, t, hh) + x) * kb[x];
+      sum += acc;
+    }
+    s.emplace_back(sum / nh_score, i);
   }
   // Highest score first; equal scores: lower block index first.
   std::sort(s.begin(), s.end(), [](const std::pair<double, int64_t>& a,
@@ -225,9 +242,11 @@ int oracle_meanpool(const void* k, int dtype, const int32_t* cu, int batch, int 
 }
 
 // Gate + top-k for every (token, q head): idx [T][Hq][topk] int32, gap [T][Hq].
-int oracle_gate_topk(const void* q, const void* k, int dtype, const int32_t* cu, int batch, int Hq,
-                     int Hkv, int d, int B, int topk, int32_t* idx, double* gap) {
-  Problem P{q, k, nullptr, dtype, cu, batch, Hq, Hkv, d, B, topk};
+int oracle_gate_topk_routed(const void* q, const void* k, int dtype, const int32_t* cu, int batch,
+                            int Hq, int Hkv, int d, int B, int topk, int routing, int32_t* idx,
+                            double* gap) {
+  Problem P{q, k, nullptr, dtype, cu, batch, Hq, Hkv, d, B, topk, routing};
+  if (routing != 0 && routing != 1) return -1;
   if (check(P)) return -1;
   for (int b = 0; b < batch; ++b)
     for (int g = 0; g < Hkv; ++g) {
@@ -249,10 +268,12 @@ int oracle_gate_topk(const void* q, const void* k, int dtype, const int32_t* cu,
 // Full forward by definition. If idx_in is non-null it supplies the chosen
 // blocks per (token, head) instead of the gate (entries outside [0, c) are
 // ignored; block c is always attended). idx_out, nkeys are optional.
-int oracle_forward(const void* q, const void* k, const void* v, int dtype, const int32_t* cu,
-                   int batch, int Hq, int Hkv, int d, int B, int topk, const int32_t* idx_in,
-                   double* out, double* lse, int32_t* idx_out, int64_t* nkeys) {
-  Problem P{q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk};
+int oracle_forward_routed(const void* q, const void* k, const void* v, int dtype,
+                          const int32_t* cu, int batch, int Hq, int Hkv, int d, int B, int topk,
+                          int routing, const int32_t* idx_in, double* out, double* lse,
+                          int32_t* idx_out, int64_t* nkeys) {
+  Problem P{q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk, routing};
+  if (routing != 0 && routing != 1) return -1;
   if (check(P)) return -1;
   for (int b = 0; b < batch; ++b)
     for (int g = 0; g < Hkv; ++g) {
@@ -283,11 +304,14 @@ int oracle_forward(const void* q, const void* k, const void* v, int dtype, const
 // writes out [nrows][d], lse [nrows], idx [nrows][topk], gap [nrows].
 // If q_rows is non-null it holds the q vectors of the listed rows ([nrows][d],
 // same dtype) and q is not read, so a caller need not hold all of q.
-int oracle_forward_rows(const void* q, const void* k, const void* v, int dtype, const int32_t* cu,
-                        int batch, int Hq, int Hkv, int d, int B, int topk, const int64_t* rows,
-                        int64_t nrows, const int32_t* idx_in, double* out, double* lse,
-                        int32_t* idx_out, double* gap, const void* q_rows) {
-  Problem P{q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk};
+int oracle_forward_rows_routed(const void* q, const void* k, const void* v, int dtype,
+                               const int32_t* cu, int batch, int Hq, int Hkv, int d, int B,
+                               int topk, int routing, const int64_t* rows, int64_t nrows,
+                               const int32_t* idx_in, double* out, double* lse, int32_t* idx_out,
+                               double* gap, const void* q_rows) {
+  Problem P{q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk, routing};
+  // shared routing reads every head of the group: not with sampled q rows
+  if ((routing != 0 && routing != 1) || (routing == 1 && q_rows)) return -1;
   if (check(P)) return -1;
   const int64_t T = batch > 0 ? cu[batch] : 0;
   for (int64_t r = 0; r < nrows; ++r)
@@ -335,6 +359,25 @@ int oracle_forward_rows(const void* q, const void* k, const void* v, int dtype, 
     attend_q(P, Pr, b, t, h, tq, hq, p, sel.data(), out + r * d, lse ? lse + r : nullptr);
   }
   return 0;
+}
+
+// Per-head routing (the default) under the original names.
+int oracle_gate_topk(const void* q, const void* k, int dtype, const int32_t* cu, int batch, int Hq,
+                     int Hkv, int d, int B, int topk, int32_t* idx, double* gap) {
+  return oracle_gate_topk_routed(q, k, dtype, cu, batch, Hq, Hkv, d, B, topk, 0, idx, gap);
+}
+int oracle_forward(const void* q, const void* k, const void* v, int dtype, const int32_t* cu,
+                   int batch, int Hq, int Hkv, int d, int B, int topk, const int32_t* idx_in,
+                   double* out, double* lse, int32_t* idx_out, int64_t* nkeys) {
+  return oracle_forward_routed(q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk, 0, idx_in, out, lse,
+                               idx_out, nkeys);
+}
+int oracle_forward_rows(const void* q, const void* k, const void* v, int dtype, const int32_t* cu,
+                        int batch, int Hq, int Hkv, int d, int B, int topk, const int64_t* rows,
+                        int64_t nrows, const int32_t* idx_in, double* out, double* lse,
+                        int32_t* idx_out, double* gap, const void* q_rows) {
+  return oracle_forward_rows_routed(q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk, 0, rows, nrows,
+                                    idx_in, out, lse, idx_out, gap, q_rows);
 }
 
 // moba_naive view: per (sequence, head) build the dense boolean mask

@@ -43,15 +43,18 @@ def index_mismatches(gpu_idx, ref_idx, gap):
     return bad
 
 
-def check_forward(q, k, v, cu, B, topk, out_gpu, lse_gpu=None, idx_gpu=None, indices=None):
+def check_forward(q, k, v, cu, B, topk, out_gpu, lse_gpu=None, idx_gpu=None, indices=None,
+                  shared_routing=False):
     """Full oracle comparison of a forward result (small shapes)."""
     dtype = q.dtype
     ref, ref_lse, ref_idx, _ = oracle.forward(q.cpu(), k.cpu(), v.cpu(), cu.cpu(), B, topk,
-                                              indices=None if indices is None else indices.cpu())
+                                              indices=None if indices is None else indices.cpu(),
+                                              shared_routing=shared_routing)
     out = out_gpu.float().cpu().numpy()
     T, Hq = q.shape[:2]
     if idx_gpu is not None and indices is None:
-        _, gap = oracle.gate_topk(q.cpu(), k.cpu(), cu.cpu(), B, topk)
+        _, gap = oracle.gate_topk(q.cpu(), k.cpu(), cu.cpu(), B, topk,
+                                  shared_routing=shared_routing)
         bad = index_mismatches(idx_gpu.cpu().numpy(), ref_idx, gap)
         if len(bad):
             # near-tie rows: the oracle with the GPU's own choice

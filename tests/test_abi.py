@@ -51,6 +51,7 @@ def test_workspace_sizes():
 
 @pytest.mark.parametrize("bad", [
     dict(num_q_heads=3, num_kv_heads=2), dict(block_size=0), dict(topk=0), dict(batch=-1),
+    dict(routing=2), dict(routing=-1),
     dict(num_kv_heads=0)])
 def test_invalid_params_rejected(bad):
     p = params(**bad)
