@@ -39,6 +39,7 @@ def _lib():
             "oracle_forward_routed": [P, P, P, I, P, I, I, I, I, I, I, I, P, P, P, P, P],
             "oracle_forward_rows_routed": [P, P, P, I, P, I, I, I, I, I, I, I, P, L, P, P, P, P, P,
                                            P],
+            "oracle_backward_routed": [P, P, P, P, I, P, I, I, I, I, I, I, I, P, P, P, P],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -152,6 +153,29 @@ def forward(q, k, v, cu_seqlens, block_size, topk, indices=None, shared_routing=
     if rc:
         raise ValueError("oracle_forward: invalid arguments")
     return out, lse, idx, nkeys
+
+
+def backward(q, k, v, dout, cu_seqlens, block_size, topk, indices=None, shared_routing=False):
+    """Gradients of sum(dout * out) by definition: (dq [T,Hq,d], dk [T,Hkv,d], dv [T,Hkv,d]),
+    float64. The block choice (a hard top-k) passes no gradient."""
+    qr, kr, vr, dt = _qkv(q, k, v)
+    dr, dd = _raw(dout)
+    if dd != dt or dr.shape != qr.shape:
+        raise TypeError("dout must have q's shape and dtype")
+    cu = _i32(cu_seqlens)
+    T, Hq, d = qr.shape
+    Hkv = kr.shape[1]
+    idx_in = None if indices is None else _i32(indices)
+    dq = np.zeros((T, Hq, d), dtype=np.float64)
+    dk = np.zeros((T, Hkv, d), dtype=np.float64)
+    dv = np.zeros((T, Hkv, d), dtype=np.float64)
+    rc = _lib().oracle_backward_routed(_ptr(qr), _ptr(kr), _ptr(vr), _ptr(dr), dt, _ptr(cu),
+                                       len(cu) - 1, Hq, Hkv, d, block_size, topk,
+                                       int(bool(shared_routing)), _ptr(idx_in), _ptr(dq), _ptr(dk),
+                                       _ptr(dv))
+    if rc:
+        raise ValueError("oracle_backward: invalid arguments")
+    return dq, dk, dv
 
 
 def forward_rows(q, k, v, cu_seqlens, block_size, topk, rows, indices=None, q_rows=None,

@@ -43,6 +43,17 @@
 // not fix the aggregate; the mean, which averages the heads' needs, is the
 // reading taken.) The *_routed entry points take routing = 0 (per head, the
 // default everywhere else) or 1 (shared by the group).
+//
+// Backward (oracle_backward_routed): gradients of L = sum(dO . O) with respect
+// to q, k and v through the chosen blocks' keys. The block choice is a hard
+// top-k and passes no gradient to the scores ([PT §5.3]: the top-k indices
+// only build the mask; the loss flows back along the Q/K/V that were read).
+// Per query row with candidate keys J, logits s_j = q.k_j / sqrt(d),
+// P_j = softmax_J(s)_j, O = sum_j P_j v_j:
+//   dP_j = dO . v_j,   D = sum_j P_j dP_j (= dO . O),   dS_j = P_j (dP_j - D)
+//   dq  = sum_j dS_j k_j / sqrt(d),  dk_j += dS_j q / sqrt(d),  dv_j += P_j dO
+// (the chain rule through the softmax; every query head adds into its kv
+// head's dk, dv).
 
 #include <algorithm>
 #include <cmath>
@@ -201,6 +212,61 @@ int64_t attend_q(const Problem& P, const Problem& Pq, int b, int64_t t, int h, i
   for (int x = 0; x < P.d; ++x) o[x] /= l;
   if (lse) *lse = m + std::log(l);
   return static_cast<int64_t>(J.size());
+}
+
+// Backward contributions of one query row (t, h) at position p of sequence b:
+// adds its dk, dv contributions to the kv head's rows of dk, dv and writes dq.
+void backward_row(const Problem& P, const void* dout, int b, int64_t t, int h, int64_t p,
+                  const int32_t* sel, double* dq, double* dk, double* dv) {
+  const int64_t start = P.cu[b];
+  const int g = h / (P.Hq / P.Hkv);
+  const int64_t c = p / P.B;
+  const double scale = 1.0 / std::sqrt(static_cast<double>(P.d));
+  std::vector<int64_t> J;
+  std::vector<int32_t> hist;
+  for (int r = 0; r < P.topk; ++r)
+    if (sel[r] >= 0 && sel[r] < c) hist.push_back(sel[r]);
+  std::sort(hist.begin(), hist.end());
+  hist.erase(std::unique(hist.begin(), hist.end()), hist.end());
+  for (int32_t i : hist)
+    for (int64_t j = static_cast<int64_t>(i) * P.B; j < static_cast<int64_t>(i + 1) * P.B; ++j)
+      J.push_back(j);
+  for (int64_t j = c * P.B; j <= p; ++j) J.push_back(j);
+  const int d = P.d;
+  std::vector<double> qv(d), dov(d);
+  for (int x = 0; x < d; ++x) {
+    qv[x] = load(P.q, P.dtype, q_off(P, t, h) + x);
+    dov[x] = load(dout, P.dtype, q_off(P, t, h) + x);
+  }
+  std::vector<double> logit(J.size()), prob(J.size()), dp(J.size());
+  double m = -std::numeric_limits<double>::infinity();
+  for (size_t r = 0; r < J.size(); ++r) {
+    double acc = 0.0;
+    for (int x = 0; x < d; ++x) acc += qv[x] * load(P.k, P.dtype, kv_off(P, start + J[r], g) + x);
+    logit[r] = acc * scale;
+    m = std::max(m, logit[r]);
+  }
+  double l = 0.0;
+  for (size_t r = 0; r < J.size(); ++r) l += (prob[r] = std::exp(logit[r] - m));
+  double D = 0.0;
+  for (size_t r = 0; r < J.size(); ++r) {
+    prob[r] /= l;
+    double acc = 0.0;
+    for (int x = 0; x < d; ++x) acc += dov[x] * load(P.v, P.dtype, kv_off(P, start + J[r], g) + x);
+    dp[r] = acc;
+    D += prob[r] * acc;
+  }
+  double* dqr = dq + q_off(P, t, h);
+  for (int x = 0; x < d; ++x) dqr[x] = 0.0;
+  for (size_t r = 0; r < J.size(); ++r) {
+    const double ds = prob[r] * (dp[r] - D);
+    const int64_t kr = kv_off(P, start + J[r], g);
+    for (int x = 0; x < d; ++x) {
+      dqr[x] += ds * scale * load(P.k, P.dtype, kr + x);
+      dk[kr + x] += ds * scale * qv[x];
+      dv[kr + x] += prob[r] * dov[x];
+    }
+  }
 }
 
 int64_t attend(const Problem& P, int b, int64_t t, int h, int64_t p, const int32_t* sel, double* o,
@@ -378,6 +444,42 @@ int oracle_forward_rows(const void* q, const void* k, const void* v, int dtype, 
                         int32_t* idx_out, double* gap, const void* q_rows) {
   return oracle_forward_rows_routed(q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk, 0, rows, nrows,
                                     idx_in, out, lse, idx_out, gap, q_rows);
+}
+
+// Backward by definition: dq [T][Hq][d], dk and dv [T][Hkv][d] (float64,
+// overwritten). dout has q's shape and dtype. If idx_in is non-null it gives
+// the chosen blocks per (token, q head), as in oracle_forward.
+int oracle_backward_routed(const void* q, const void* k, const void* v, const void* dout, int dtype,
+                           const int32_t* cu, int batch, int Hq, int Hkv, int d, int B, int topk,
+                           int routing, const int32_t* idx_in, double* dq, double* dk,
+                           double* dv) {
+  Problem P{q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk, routing};
+  if (check(P) || (routing != 0 && routing != 1) || !dout) return -1;
+  const int64_t T = batch > 0 ? cu[batch] : 0;
+  std::fill(dk, dk + T * Hkv * d, 0.0);
+  std::fill(dv, dv + T * Hkv * d, 0.0);
+  const int grp = Hq / Hkv;
+  // one (sequence, kv head) per task: it alone writes that kv head's dk, dv
+  // rows and its query heads' dq rows
+#pragma omp parallel for schedule(dynamic)
+  for (int64_t bg = 0; bg < static_cast<int64_t>(batch) * Hkv; ++bg) {
+    const int b = static_cast<int>(bg / Hkv), g = static_cast<int>(bg % Hkv);
+    std::vector<double> kb;
+    if (!idx_in) block_means(P, b, g, kb);
+    const int64_t len = cu[b + 1] - cu[b];
+    std::vector<int32_t> sel(static_cast<size_t>(topk));
+    for (int64_t p = 0; p < len; ++p)
+      for (int hh = 0; hh < grp; ++hh) {
+        const int h = g * grp + hh;
+        const int64_t t = cu[b] + p;
+        if (idx_in)
+          std::memcpy(sel.data(), idx_in + (t * Hq + h) * topk, sizeof(int32_t) * topk);
+        else
+          select_blocks(P, t, h, p, kb, sel.data(), nullptr);
+        backward_row(P, dout, b, t, h, p, sel.data(), dq, dk, dv);
+      }
+  }
+  return 0;
 }
 
 // moba_naive view: per (sequence, head) build the dense boolean mask
