@@ -163,6 +163,29 @@ MOBA_API moba_status moba_forward_with_indices(const moba_params* p, const void*
                                       const int32_t* idx, void* out, float* lse, void* ws,
                                       size_t ws_bytes, void* stream);
 
+/* Backward pass (PaperTrace "2.1.3 MoBA", section 5.3: the hard top-k
+ * indices only build the mask and pass no gradient to the routing scores;
+ * the loss flows back through the Q/K/V that were read). Gradients of
+ * L = sum(dout * out) with respect to q, k and v over the same candidate keys
+ * as the forward: per query row, P_j = exp(q.k_j / sqrt(d) - lse),
+ * dS_j = P_j (dout.v_j - dout.out), dq = sum_j dS_j k_j / sqrt(d),
+ * dk_j += dS_j q / sqrt(d), dv_j += P_j dout (every q head of a group adds
+ * into its kv head's dk, dv).
+ *   q, k, v, cu_seqlens: as for moba_forward; out [T][Hq][d] and lse [T][Hq]
+ *   (fp32, natural log): the forward's results for these inputs; dout:
+ *   [T][Hq][d], q's dtype.
+ *   idx: the forward's index rows [T][Hq][k] (canonical form), or NULL to
+ *   run the gate again (p->routing as in the forward).
+ *   dq [T][Hq][d], dk and dv [T][Hkv][d]: fp32, caller-owned, overwritten.
+ *   ws: moba_backward_workspace_size(p, idx != NULL) bytes, 16-byte aligned.
+ * Errors as moba_forward (MOBA_ERR_BAD_INDICES via the status word). */
+MOBA_API size_t moba_backward_workspace_size(const moba_params* p, int have_indices);
+MOBA_API moba_status moba_backward(const moba_params* p, const void* q, const void* k,
+                                   const void* v, const int32_t* cu_seqlens, const void* out,
+                                   const float* lse, const void* dout, const int32_t* idx,
+                                   float* dq, float* dk, float* dv, void* ws, size_t ws_bytes,
+                                   void* stream);
+
 /* Dense causal softmax attention, eq. (1) with a causal mask (every key
  * j <= p of the query's own sequence), for comparison and for the full
  * budget limit (section 4). block_size and topk in p must be valid but do

@@ -194,6 +194,33 @@ def moba_forward(q, k, v, cu_seqlens, block_size: int, topk: int, max_seqlen=Non
     return (out, lse) if return_lse else out
 
 
+def moba_backward(q, k, v, cu_seqlens, out, lse, dout, block_size: int, topk: int,
+                  idx: Optional[torch.Tensor] = None, max_seqlen=None,
+                  shared_routing: bool = False):
+    """Gradients of sum(dout * out) through the chosen blocks: (dq [T,Hq,d], dk, dv [T,Hkv,d])
+    in fp32. out, lse: the forward's results; idx: its index rows, or None to run the gate
+    again."""
+    _check_inputs(q, k, v, out, dout, lse, idx)
+    L = lib()
+    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen, shared_routing)
+    cu = _dev_i32(cu_seqlens, q.device)
+    L.moba_backward_workspace_size.argtypes = [ctypes.POINTER(MobaParams), ctypes.c_int]
+    L.moba_backward_workspace_size.restype = ctypes.c_size_t
+    nbytes = int(L.moba_backward_workspace_size(ctypes.byref(p), 0 if idx is None else 1))
+    ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    fn = L.moba_backward
+    fn.argtypes = [ctypes.POINTER(MobaParams)] + [ctypes.c_void_p] * 12 + [ctypes.c_size_t,
+                                                                         ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check("moba_backward", fn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(cu), _ptr(out),
+                               _ptr(lse), _ptr(dout), _ptr(idx), _ptr(dq), _ptr(dk), _ptr(dv),
+                               _ptr(ws), ws.numel(), _stream(q.device)))
+    return dq, dk, dv
+
+
 def moba_forward_with_indices(q, k, v, cu_seqlens, idx, block_size: int, max_seqlen=None,
                               return_lse: bool = False, ws: Optional[torch.Tensor] = None):
     """MoBA forward with caller-chosen blocks idx int32 [T, Hq, topk] (canonical form)."""

@@ -204,6 +204,88 @@ moba_status forward_impl(const moba_params* p, const void* q, const void* k, con
   return MOBA_OK;
 }
 
+// Backward workspace: block means and index rows when the gate runs again,
+// the regroup lists of every kv head (one pass), and D = dO . O per row.
+struct BwdLayout {
+  size_t kbar, idx, counts, cursor, list_off, tile_off, pairs, tiles, dsum, total;
+  int64_t max_tiles;
+};
+
+BwdLayout plan_bwd(const Dims& dm, bool own_idx) {
+  BwdLayout L{};
+  const int64_t n_lists = (int64_t)dm.batch * dm.Hkv * dm.nb;
+  const int64_t max_pairs = (int64_t)dm.T * dm.Hq * (dm.topk - 1);
+  L.max_tiles = (max_pairs + kSimtTileM - 1) / kSimtTileM + n_lists;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L.kbar = take(own_idx ? sizeof(float) * (size_t)dm.batch * dm.nb * dm.Hkv * dm.d : 0);
+  L.idx = take(own_idx ? sizeof(int32_t) * (size_t)dm.T * dm.Hq * dm.topk : 0);
+  L.counts = take(sizeof(int32_t) * n_lists);
+  L.cursor = take(sizeof(int32_t) * n_lists);
+  L.list_off = take(sizeof(int32_t) * (n_lists + 1));
+  L.tile_off = take(sizeof(int32_t) * (n_lists + 1));
+  L.pairs = take(sizeof(int32_t) * max_pairs);
+  L.tiles = take(sizeof(int2) * L.max_tiles);
+  L.dsum = take(sizeof(float) * (size_t)dm.T * dm.Hq);
+  L.total = off;
+  return L;
+}
+
+moba_status backward_impl(const moba_params* p, const void* q, const void* k, const void* v,
+                          const int32_t* cu, const void* out, const float* lse, const void* dout,
+                          const int32_t* idx_in, float* dq, float* dk, float* dv, void* ws,
+                          size_t ws_bytes, void* stream) {
+  Dims dm;
+  moba_status s = validate(p, dm);
+  if (s != MOBA_OK) return s;
+  if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
+  if (!q || !k || !v || !cu || !out || !lse || !dout || !dq || !dk || !dv)
+    return MOBA_ERR_INVALID_ARG;
+  for (const void* x : {q, k, v, out, dout, static_cast<const void*>(dq),
+                        static_cast<const void*>(dk), static_cast<const void*>(dv)})
+    if (!aligned16(x)) return MOBA_ERR_INVALID_ARG;
+  const BwdLayout L = plan_bwd(dm, idx_in == nullptr);
+  if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOBA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = status_word();
+  if (!status) return MOBA_ERR_CUDA;
+  char* base = static_cast<char*>(ws);
+  MOBA_TRY(cudaMemsetAsync(dq, 0, sizeof(float) * (size_t)dm.T * dm.Hq * dm.d, st));
+  MOBA_TRY(cudaMemsetAsync(dk, 0, sizeof(float) * (size_t)dm.T * dm.Hkv * dm.d, st));
+  MOBA_TRY(cudaMemsetAsync(dv, 0, sizeof(float) * (size_t)dm.T * dm.Hkv * dm.d, st));
+  const int32_t* idx = idx_in;
+  if (!idx_in) {
+    float* kbar = reinterpret_cast<float*>(base + L.kbar);
+    int32_t* own = reinterpret_cast<int32_t*>(base + L.idx);
+    MOBA_TRY(launch_meanpool(dm, k, cu, kbar, status, st));
+    MOBA_TRY(launch_gate(dm, q, kbar, cu, own, status, st));
+    idx = own;
+  }
+  Regroup rg;
+  rg.counts = reinterpret_cast<int32_t*>(base + L.counts);
+  rg.cursor = reinterpret_cast<int32_t*>(base + L.cursor);
+  rg.list_off = reinterpret_cast<int32_t*>(base + L.list_off);
+  rg.tile_off = reinterpret_cast<int32_t*>(base + L.tile_off);
+  rg.pairs = reinterpret_cast<int32_t*>(base + L.pairs);
+  rg.tiles = reinterpret_cast<int2*>(base + L.tiles);
+  rg.max_tiles = L.max_tiles;
+  Chunk ch;
+  ch.g0 = 0;
+  ch.ng = dm.Hkv;
+  ch.h0 = 0;
+  ch.nq = dm.Hq;
+  ch.n_lists = dm.batch * dm.Hkv * dm.nb;
+  ch.tile_m = kSimtTileM;
+  MOBA_TRY(launch_regroup(dm, ch, idx, cu, rg, status, st));
+  MOBA_TRY(launch_backward(dm, ch, q, k, v, out, dout, lse, reinterpret_cast<float*>(base + L.dsum),
+                           cu, rg, dq, dk, dv, status, st));
+  return MOBA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -212,6 +294,20 @@ int moba_num_blocks(const moba_params* p) {
   Dims dm;
   if (validate(p, dm) != MOBA_OK) return 0;
   return dm.nb;
+}
+
+size_t moba_backward_workspace_size(const moba_params* p, int have_indices) {
+  Dims dm;
+  if (validate(p, dm) != MOBA_OK) return 0;
+  return plan_bwd(dm, have_indices == 0).total;
+}
+
+moba_status moba_backward(const moba_params* p, const void* q, const void* k, const void* v,
+                          const int32_t* cu_seqlens, const void* out, const float* lse,
+                          const void* dout, const int32_t* idx, float* dq, float* dk, float* dv,
+                          void* ws, size_t ws_bytes, void* stream) {
+  return backward_impl(p, q, k, v, cu_seqlens, out, lse, dout, idx, dq, dk, dv, ws, ws_bytes,
+                       stream);
 }
 
 size_t moba_workspace_size(const moba_params* p) {
