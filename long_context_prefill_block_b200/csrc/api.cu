@@ -281,8 +281,12 @@ moba_status backward_impl(const moba_params* p, const void* q, const void* k, co
   ch.n_lists = dm.batch * dm.Hkv * dm.nb;
   ch.tile_m = kSimtTileM;
   MOBA_TRY(launch_regroup(dm, ch, idx, cu, rg, status, st));
-  MOBA_TRY(launch_backward(dm, ch, q, k, v, out, dout, lse, reinterpret_cast<float*>(base + L.dsum),
-                           cu, rg, dq, dk, dv, status, st));
+  float* dsum = reinterpret_cast<float*>(base + L.dsum);
+  MOBA_TRY(launch_bwd_dot(dm, out, dout, dsum, st));
+  if (bwd_tc_supported(dm))
+    MOBA_TRY(launch_backward_tc(dm, ch, q, k, v, dout, lse, dsum, cu, rg, dq, dk, dv, status, st));
+  else
+    MOBA_TRY(launch_backward(dm, ch, q, k, v, dout, lse, dsum, cu, rg, dq, dk, dv, status, st));
   return MOBA_OK;
 }
 

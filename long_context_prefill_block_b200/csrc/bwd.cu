@@ -281,15 +281,19 @@ __global__ void __launch_bounds__(kThreads) bwd_block_kernel(const BwdArgs a) {
 }
 
 template <typename T, int D>
-cudaError_t run(const BwdArgs& a, const void* out, int n_lists, cudaStream_t st) {
+cudaError_t run_dot(const Dims& dm, const void* out, const void* dout, float* Dsum,
+                    cudaStream_t st) {
+  const int64_t rows = (int64_t)dm.T * dm.Hq;
+  if (rows <= 0) return cudaSuccess;
+  bwd_dot_kernel<T, D><<<(unsigned)((rows + 7) / 8), kThreads, 0, st>>>(
+      rows, static_cast<const T*>(dout), static_cast<const T*>(out), Dsum);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t run(const BwdArgs& a, int n_lists, cudaStream_t st) {
   const Dims& dm = a.dm;
   cudaError_t e;
-  const int64_t rows = (int64_t)dm.T * dm.Hq;
-  if (rows > 0) {
-    bwd_dot_kernel<T, D><<<(unsigned)((rows + 7) / 8), kThreads, 0, st>>>(
-        rows, static_cast<const T*>(a.dout), static_cast<const T*>(out), const_cast<float*>(a.Dsum));
-    if ((e = cudaGetLastError())) return e;
-  }
   const size_t smem = BwdSmem<D>::bytes;
   if ((e = cudaFuncSetAttribute(bwd_block_kernel<T, D, HIST>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
@@ -312,10 +316,19 @@ cudaError_t run(const BwdArgs& a, const void* out, int n_lists, cudaStream_t st)
 
 }  // namespace
 
+cudaError_t launch_bwd_dot(const Dims& dm, const void* out, const void* dout, float* Dsum,
+                           cudaStream_t st) {
+  if (dm.dtype == kBF16)
+    return dm.d == 128 ? run_dot<__nv_bfloat16, 128>(dm, out, dout, Dsum, st)
+                       : run_dot<__nv_bfloat16, 64>(dm, out, dout, Dsum, st);
+  return dm.d == 128 ? run_dot<float, 128>(dm, out, dout, Dsum, st)
+                     : run_dot<float, 64>(dm, out, dout, Dsum, st);
+}
+
 cudaError_t launch_backward(const Dims& dm, const Chunk& ch, const void* q, const void* k,
-                            const void* v, const void* out, const void* dout, const float* lse,
-                            float* Dsum, const int32_t* cu, const Regroup& rg, float* dq,
-                            float* dk, float* dv, int* status, cudaStream_t st) {
+                            const void* v, const void* dout, const float* lse, const float* Dsum,
+                            const int32_t* cu, const Regroup& rg, float* dq, float* dk, float* dv,
+                            int* status, cudaStream_t st) {
   if (dm.batch == 0 || dm.max_seqlen == 0) return cudaSuccess;
   BwdArgs a{};
   a.dm = dm;
@@ -334,10 +347,10 @@ cudaError_t launch_backward(const Dims& dm, const Chunk& ch, const void* q, cons
   a.dv = dv;
   a.status = status;
   if (dm.dtype == kBF16)
-    return dm.d == 128 ? run<__nv_bfloat16, 128>(a, out, ch.n_lists, st)
-                       : run<__nv_bfloat16, 64>(a, out, ch.n_lists, st);
-  return dm.d == 128 ? run<float, 128>(a, out, ch.n_lists, st)
-                     : run<float, 64>(a, out, ch.n_lists, st);
+    return dm.d == 128 ? run<__nv_bfloat16, 128>(a, ch.n_lists, st)
+                       : run<__nv_bfloat16, 64>(a, ch.n_lists, st);
+  return dm.d == 128 ? run<float, 128>(a, ch.n_lists, st)
+                     : run<float, 64>(a, ch.n_lists, st);
 }
 
 }  // namespace moba

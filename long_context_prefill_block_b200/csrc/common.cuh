@@ -138,10 +138,18 @@ cudaError_t launch_dense_simt(const Dims& dm, const void* q, const void* k, cons
                               const int32_t* cu, void* out, float* lse, cudaStream_t st);
 // Backward (bwd.cu): dq, dk, dv (fp32, zeroed by the caller) of the whole
 // batch; `ch` covers every head in one pass; Dsum [T * Hq] is scratch.
+cudaError_t launch_bwd_dot(const Dims& dm, const void* out, const void* dout, float* Dsum,
+                           cudaStream_t st);
 cudaError_t launch_backward(const Dims& dm, const Chunk& ch, const void* q, const void* k,
-                            const void* v, const void* out, const void* dout, const float* lse,
-                            float* Dsum, const int32_t* cu, const Regroup& rg, float* dq,
-                            float* dk, float* dv, int* status, cudaStream_t st);
+                            const void* v, const void* dout, const float* lse, const float* Dsum,
+                            const int32_t* cu, const Regroup& rg, float* dq, float* dk, float* dv,
+                            int* status, cudaStream_t st);
+// Tensor-core backward (bf16, d = 128, B % 128 == 0).
+bool bwd_tc_supported(const Dims& dm);
+cudaError_t launch_backward_tc(const Dims& dm, const Chunk& ch, const void* q, const void* k,
+                               const void* v, const void* dout, const float* lse,
+                               const float* Dsum, const int32_t* cu, const Regroup& rg,
+                               float* dq, float* dk, float* dv, int* status, cudaStream_t st);
 constexpr int kSimtTileM = 32;
 
 cudaError_t launch_merge(const Dims& dm, const Chunk& ch, const int32_t* idx, const int32_t* cu,
