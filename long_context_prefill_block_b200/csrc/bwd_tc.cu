@@ -72,6 +72,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ C
   __shared__ uint64_t kv_full, mma_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
+  __shared__ int64_t qrow_s[TM];
+  __shared__ int pos_s[TM];
   const Dims& dm = a.dm;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int grp = dm.Hq / dm.Hkv;
@@ -254,16 +256,48 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ C
     ++nmma;
     if (!__syncthreads_and(ok)) { ok = false; break; }
     fence_after_sync();
-    // ---- dq of row r (every lane takes part in the warp's TMEM loads)
+    // ---- dq: rows through shared memory (the P and dS tiles are free now:
+    // their MMAs are done), then each warp adds whole 512-byte rows with
+    // 16-byte vector reductions. Row r's 16-byte chunk c sits at chunk
+    // c ^ (r % 32) of its row, so neither side has bank conflicts beyond the
+    // four wavefronts a 512-byte access needs.
+    {
+      const uint32_t st = sbase + kP;  // 128 rows x 512 bytes = the P and dS tiles
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t v[32];
-      tmem_ld32(tmem + 0 + lane_addr + c * 32, v);
-      tmem_wait_ld();
-      if (pos >= 0) {
-        float* dst = a.dq + qrow * D + c * 32;
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + 0 + lane_addr + c * 32, v);
+        tmem_wait_ld();
 #pragma unroll
-        for (int x = 0; x < 32; ++x) atomicAdd(dst + x, __uint_as_float(v[x]) * scale);
+        for (int x4 = 0; x4 < 8; ++x4) {
+          const uint32_t chunk = (uint32_t)(c * 8 + x4) ^ ((uint32_t)r & 31u);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(st + r * 512 + chunk * 16),
+                       "r"(__float_as_uint(__uint_as_float(v[4 * x4]) * scale)),
+                       "r"(__float_as_uint(__uint_as_float(v[4 * x4 + 1]) * scale)),
+                       "r"(__float_as_uint(__uint_as_float(v[4 * x4 + 2]) * scale)),
+                       "r"(__float_as_uint(__uint_as_float(v[4 * x4 + 3]) * scale))
+                       : "memory");
+        }
+      }
+      qrow_s[r] = qrow;
+      pos_s[r] = pos;
+      __syncthreads();
+      const int lane = tid & 31;
+#pragma unroll 4
+      for (int i = 0; i < TM / 4; ++i) {
+        const int row = warp * (TM / 4) + i;
+        if (pos_s[row] < 0) continue;  // warp-uniform
+        const uint32_t chunk = (uint32_t)lane ^ ((uint32_t)row & 31u);
+        uint32_t x, y, z, w;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(x), "=r"(y), "=r"(z), "=r"(w)
+                     : "r"(st + row * 512 + chunk * 16)
+                     : "memory");
+        float* dst = a.dq + qrow_s[row] * D + lane * 4;
+        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst),
+                     "f"(__uint_as_float(x)), "f"(__uint_as_float(y)), "f"(__uint_as_float(z)),
+                     "f"(__uint_as_float(w))
+                     : "memory");
       }
     }
     fence_before_sync();
