@@ -139,41 +139,50 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ C
   bool ok = __syncthreads_and(mbar_wait(&kv_full, 0, abort, status));
   uint32_t nmma = 0;
 
-  for (int64_t c0 = 0; ok && c0 < n_rows; c0 += TM) {
-    // ---- rows of this tile: q row ids, positions, lse and D
-    const int r = tid;
-    float lse_r = 0.f, d_r = 0.f;
-    int pos = -1;
-    int64_t qrow = 0;
-    {
-      const int64_t i = c0 + r;
-      if (i < n_rows) {
-        if (MODE == HIST) {
-          const int64_t prow = a.pairs[row0 + i];
-          const int64_t th = prow / dm.topk;
-          qrow = (th / a.ch.nq) * dm.Hq + a.ch.h0 + (int)(th % a.ch.nq);
-          pos = 0;
-        } else {
-          const int p = p_first + (int)(i / grp);
-          qrow = (start + p) * dm.Hq + g * grp + (int)(i % grp);
-          pos = p;
-        }
-        lse_r = a.lse[qrow];
-        d_r = a.Dsum[qrow];
+  // Row metadata of a tile (q row id, position, lse, D) and the cp.async of
+  // its Q and dO rows. The next tile's metadata is read while the current
+  // tile's MMAs run, and its rows are requested as soon as the Q / dO
+  // buffers are free, so both latencies hide behind the current tile.
+  const int r = tid;
+  auto meta = [&](int64_t c0, int64_t& qrow, int& pos, float& lse_r, float& d_r) {
+    const int64_t i = c0 + r;
+    qrow = 0;
+    pos = -1;
+    lse_r = d_r = 0.f;
+    if (i < n_rows) {
+      if (MODE == HIST) {
+        const int64_t th = a.pairs[row0 + i] / dm.topk;
+        qrow = (th / a.ch.nq) * dm.Hq + a.ch.h0 + (int)(th % a.ch.nq);
+        pos = 0;
+      } else {
+        const int p = p_first + (int)(i / grp);
+        qrow = (start + p) * dm.Hq + g * grp + (int)(i % grp);
+        pos = p;
       }
+      lse_r = a.lse[qrow];
+      d_r = a.Dsum[qrow];
     }
-    // ---- Q and dO rows (gathered), zero-filled past the last row
-    {
-      const __nv_bfloat16* qs = a.q + (pos >= 0 ? qrow : 0) * (int64_t)D;
-      const __nv_bfloat16* os = a.dout + (pos >= 0 ? qrow : 0) * (int64_t)D;
+  };
+  auto request = [&](int64_t qrow, int pos) {
+    const __nv_bfloat16* qs = a.q + (pos >= 0 ? qrow : 0) * (int64_t)D;
+    const __nv_bfloat16* os = a.dout + (pos >= 0 ? qrow : 0) * (int64_t)D;
 #pragma unroll
-      for (int c16 = 0; c16 < 16; ++c16) {
-        cp_async16(swz(sbase + kQ, r, c16), qs + c16 * 8, pos >= 0 ? 16u : 0u);
-        cp_async16(swz(sbase + kO, r, c16), os + c16 * 8, pos >= 0 ? 16u : 0u);
-      }
-      cp_async_wait_all();
-      fence_proxy_async_smem();
+    for (int c16 = 0; c16 < 16; ++c16) {
+      cp_async16(swz(sbase + kQ, r, c16), qs + c16 * 8, pos >= 0 ? 16u : 0u);
+      cp_async16(swz(sbase + kO, r, c16), os + c16 * 8, pos >= 0 ? 16u : 0u);
     }
+  };
+  int64_t qrow_n;
+  int pos_n;
+  float lse_n, d_n;
+  meta(0, qrow_n, pos_n, lse_n, d_n);
+  if (ok) request(qrow_n, pos_n);
+  for (int64_t c0 = 0; ok && c0 < n_rows; c0 += TM) {
+    const int64_t qrow = qrow_n;
+    const int pos = pos_n;
+    const float lse_r = lse_n, d_r = d_n;
+    cp_async_wait_all();
+    fence_proxy_async_smem();
     fence_before_sync();
     __syncthreads();
     // ---- S = Q K^T, dP = dO V^T
@@ -252,10 +261,14 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ C
       }
       commit(&mma_bar);
     }
+    const bool more = c0 + TM < n_rows;
+    if (more) meta(c0 + TM, qrow_n, pos_n, lse_n, d_n);
     ok = mbar_wait(&mma_bar, nmma & 1, abort, status);
     ++nmma;
     if (!__syncthreads_and(ok)) { ok = false; break; }
     fence_after_sync();
+    // the Q and dO buffers are free: the next tile's rows may land
+    if (more) request(qrow_n, pos_n);
     // ---- dq: rows through shared memory (the P and dS tiles are free now:
     // their MMAs are done), then each warp adds whole 512-byte rows with
     // 16-byte vector reductions. Row r's 16-byte chunk c sits at chunk
@@ -303,6 +316,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ C
     fence_before_sync();
     __syncthreads();
   }
+  cp_async_wait_all();  // an early exit may leave the next tile's rows in flight
   // ---- dK, dV of key k0 + tid (TMEM lane tid)
   if (ok) {
     const int key = k0 + tid;
