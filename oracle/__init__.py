@@ -40,6 +40,7 @@ def _lib():
             "oracle_forward_rows_routed": [P, P, P, I, P, I, I, I, I, I, I, I, P, L, P, P, P, P, P,
                                            P],
             "oracle_backward_routed": [P, P, P, P, I, P, I, I, I, I, I, I, I, P, P, P, P],
+            "oracle_forward_mask_routed": [P, P, P, I, P, I, I, I, I, I, I, I, P, P],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -86,6 +87,13 @@ def _i32(x):
     return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
 
 
+def _routing(shared_routing, prefix_mean):
+    """Routing flags of the *_routed entry points: bit 0 = one choice per kv
+    head's group (the group's mean score), bit 1 = the own block scored by the
+    mean of its keys up to the query instead of forced."""
+    return int(bool(shared_routing)) | (int(bool(prefix_mean)) << 1)
+
+
 def _ptr(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
@@ -118,10 +126,11 @@ def meanpool(k, cu_seqlens, block_size):
     return out
 
 
-def gate_topk(q, k, cu_seqlens, block_size, topk, shared_routing=False):
+def gate_topk(q, k, cu_seqlens, block_size, topk, shared_routing=False, prefix_mean=False):
     """(idx [T, Hq, topk] int32, gap [T, Hq] float64). shared_routing: every
     query head of a kv head's group takes the blocks chosen by the group's
-    mean score."""
+    mean score. prefix_mean: the own block is scored by the mean of its keys
+    up to the query and competes for the k slots instead of being forced."""
     qr, kr, _, dt = _qkv(q, k, None)
     cu = _i32(cu_seqlens)
     T, Hq, d = qr.shape
@@ -129,14 +138,16 @@ def gate_topk(q, k, cu_seqlens, block_size, topk, shared_routing=False):
     idx = np.full((T, Hq, topk), -1, dtype=np.int32)
     gap = np.zeros((T, Hq), dtype=np.float64)
     rc = _lib().oracle_gate_topk_routed(_ptr(qr), _ptr(kr), dt, _ptr(cu), len(cu) - 1, Hq, Hkv, d,
-                                        block_size, topk, int(bool(shared_routing)), _ptr(idx),
+                                        block_size, topk, _routing(shared_routing, prefix_mean),
+                                        _ptr(idx),
                                         _ptr(gap))
     if rc:
         raise ValueError("oracle_gate_topk: invalid arguments")
     return idx, gap
 
 
-def forward(q, k, v, cu_seqlens, block_size, topk, indices=None, shared_routing=False):
+def forward(q, k, v, cu_seqlens, block_size, topk, indices=None, shared_routing=False,
+            prefix_mean=False):
     """Full forward by definition: (out [T,Hq,d], lse [T,Hq], idx [T,Hq,topk], nkeys [T,Hq])."""
     qr, kr, vr, dt = _qkv(q, k, v)
     cu = _i32(cu_seqlens)
@@ -148,14 +159,15 @@ def forward(q, k, v, cu_seqlens, block_size, topk, indices=None, shared_routing=
     idx = np.full((T, Hq, topk), -1, dtype=np.int32)
     nkeys = np.zeros((T, Hq), dtype=np.int64)
     rc = _lib().oracle_forward_routed(_ptr(qr), _ptr(kr), _ptr(vr), dt, _ptr(cu), len(cu) - 1, Hq,
-                                      Hkv, d, block_size, topk, int(bool(shared_routing)),
-                                      _ptr(idx_in), _ptr(out), _ptr(lse), _ptr(idx), _ptr(nkeys))
+                                      Hkv, d, block_size, topk,
+                                      _routing(shared_routing, prefix_mean), _ptr(idx_in), _ptr(out), _ptr(lse), _ptr(idx), _ptr(nkeys))
     if rc:
         raise ValueError("oracle_forward: invalid arguments")
     return out, lse, idx, nkeys
 
 
-def backward(q, k, v, dout, cu_seqlens, block_size, topk, indices=None, shared_routing=False):
+def backward(q, k, v, dout, cu_seqlens, block_size, topk, indices=None, shared_routing=False,
+             prefix_mean=False):
     """Gradients of sum(dout * out) by definition: (dq [T,Hq,d], dk [T,Hkv,d], dv [T,Hkv,d]),
     float64. The block choice (a hard top-k) passes no gradient."""
     qr, kr, vr, dt = _qkv(q, k, v)
@@ -171,7 +183,8 @@ def backward(q, k, v, dout, cu_seqlens, block_size, topk, indices=None, shared_r
     dv = np.zeros((T, Hkv, d), dtype=np.float64)
     rc = _lib().oracle_backward_routed(_ptr(qr), _ptr(kr), _ptr(vr), _ptr(dr), dt, _ptr(cu),
                                        len(cu) - 1, Hq, Hkv, d, block_size, topk,
-                                       int(bool(shared_routing)), _ptr(idx_in), _ptr(dq), _ptr(dk),
+                                       _routing(shared_routing, prefix_mean), _ptr(idx_in), _ptr(dq),
+                                       _ptr(dk),
                                        _ptr(dv))
     if rc:
         raise ValueError("oracle_backward: invalid arguments")
@@ -179,7 +192,7 @@ def backward(q, k, v, dout, cu_seqlens, block_size, topk, indices=None, shared_r
 
 
 def forward_rows(q, k, v, cu_seqlens, block_size, topk, rows, indices=None, q_rows=None,
-                 num_q_heads=None, shared_routing=False):
+                 num_q_heads=None, shared_routing=False, prefix_mean=False):
     """Sampled forward on rows (row = t*Hq + h): (out [n,d], lse [n], idx [n,topk], gap [n]).
 
     With q_rows ([n, d], the q vectors of the listed rows) q may be None and
@@ -208,7 +221,8 @@ def forward_rows(q, k, v, cu_seqlens, block_size, topk, rows, indices=None, q_ro
     gap = np.zeros(n, dtype=np.float64)
     rc = _lib().oracle_forward_rows_routed(_ptr(qbase), _ptr(kr), _ptr(vr), dt, _ptr(cu),
                                            len(cu) - 1, Hq, Hkv, d, block_size, topk,
-                                           int(bool(shared_routing)), _ptr(rows), n, _ptr(idx_in),
+                                           _routing(shared_routing, prefix_mean), _ptr(rows), n,
+                                           _ptr(idx_in),
                                            _ptr(out), _ptr(lse), _ptr(idx), _ptr(gap),
                                            _ptr(qr) if q_rows is not None else None)
     if rc:
@@ -216,7 +230,7 @@ def forward_rows(q, k, v, cu_seqlens, block_size, topk, rows, indices=None, q_ro
     return out, lse, idx, gap
 
 
-def forward_mask(q, k, v, cu_seqlens, block_size, topk, indices=None):
+def forward_mask(q, k, v, cu_seqlens, block_size, topk, indices=None, prefix_mean=False):
     """moba_naive view: dense boolean mask + masked dense softmax. out [T,Hq,d]."""
     qr, kr, vr, dt = _qkv(q, k, v)
     cu = _i32(cu_seqlens)
@@ -224,8 +238,9 @@ def forward_mask(q, k, v, cu_seqlens, block_size, topk, indices=None):
     Hkv = kr.shape[1]
     idx_in = None if indices is None else _i32(indices)
     out = np.zeros((T, Hq, d), dtype=np.float64)
-    rc = _lib().oracle_forward_mask(_ptr(qr), _ptr(kr), _ptr(vr), dt, _ptr(cu), len(cu) - 1, Hq,
-                                    Hkv, d, block_size, topk, _ptr(idx_in), _ptr(out))
+    rc = _lib().oracle_forward_mask_routed(_ptr(qr), _ptr(kr), _ptr(vr), dt, _ptr(cu), len(cu) - 1,
+                                           Hq, Hkv, d, block_size, topk, _routing(False, prefix_mean),
+                                           _ptr(idx_in), _ptr(out))
     if rc:
         raise ValueError("oracle_forward_mask: invalid arguments")
     return out

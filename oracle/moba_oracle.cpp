@@ -41,8 +41,23 @@
 //   s_i = (1/grp) sum_{h in group} q_{p,h} . kbar_i
 // under the same causal mask, forced own block and tie rule. (The pages do
 // not fix the aggregate; the mean, which averages the heads' needs, is the
-// reading taken.) The *_routed entry points take routing = 0 (per head, the
-// default everywhere else) or 1 (shared by the group).
+// reading taken.)
+//
+// Own-block variant ([PT §5.2], the paragraph on causal blocks: the own
+// block's full mean would include keys after the query, so a correct gate
+// either scores the own block by the mean of its keys up to the query -- the
+// prefix mean -- or forces it in unscored; the forced branch is the default
+// above). With the prefix mean, block c competes with the earlier blocks on
+//   s_c = q_p . (1/(p - cB + 1)) sum_{j=cB..p} k_j
+// and the k slots go to the best min(k, c+1) of blocks 0..c (ties to the lower
+// index, so block c loses a tie). If block c is not chosen the query reads no
+// key of its own block -- not even itself -- and its softmax runs over the
+// chosen earlier blocks only (never empty: c = 0 leaves block 0 as the one
+// candidate). With shared routing the group's mean of s_c is used.
+//
+// The *_routed entry points take routing as bit flags: bit 0 = shared by the
+// group (0: per head, the default everywhere else), bit 1 = own block scored
+// by its prefix mean (0: forced).
 //
 // Backward (oracle_backward_routed): gradients of L = sum(dO . O) with respect
 // to q, k and v through the chosen blocks' keys. The block choice is a hard
@@ -77,7 +92,10 @@ struct Problem {
   const int32_t* cu;  // [batch + 1]
   int batch, Hq, Hkv, d, B, topk;
   int shared;  // 1: the kv head's query heads share their blocks (mean score)
+  int prefix;  // 1: the own block is scored by its prefix mean, not forced
 };
+
+bool routing_ok(int routing) { return routing >= 0 && routing <= 3; }
 
 // Exact widening of a stored element to double.
 inline double load(const void* p, int dtype, int64_t i) {
@@ -128,23 +146,34 @@ void block_means(const Problem& P, int b, int g, std::vector<double>& kbar) {
 // Gate for one query: [PT §1 eq.3, §2, §2.1]. Writes the chosen blocks in
 // ascending order (history first, then the current block c) padded with -1,
 // and the relative score gap between the worst chosen and the best rejected
-// history block (infinity when nothing was left out).
+// candidate (infinity when nothing was left out). With P.prefix the own block
+// is a scored candidate ([PT §5.2]) and may be left out; its keys are read at
+// token kt (the query's token) of kv head g.
 void select_blocks(const Problem& P, int64_t t, int h, int64_t p, const std::vector<double>& kbar,
-                   int32_t* sel, double* gap) {
+                   int32_t* sel, double* gap, int64_t kt, int g) {
   const int64_t c = p / P.B;
   std::vector<std::pair<double, int64_t>> s;
-  s.reserve(static_cast<size_t>(c));
+  s.reserve(static_cast<size_t>(c + 1));
   const int grp = P.Hq / P.Hkv;
   const int h0 = P.shared ? (h / grp) * grp : h, nh_score = P.shared ? grp : 1;
-  for (int64_t i = 0; i < c; ++i) {
-    const double* kb = &kbar[static_cast<size_t>(i * P.d)];
+  auto score = [&](const double* kb) {
     double sum = 0.0;
     for (int hh = h0; hh < h0 + nh_score; ++hh) {
       double acc = 0.0;
       for (int x = 0; x < P.d; ++x) acc += load(P.q, P.dtype, q_off(P, t, hh) + x) * kb[x];
       sum += acc;
     }
-    s.emplace_back(sum / nh_score, i);
+    return sum / nh_score;
+  };
+  for (int64_t i = 0; i < c; ++i) s.emplace_back(score(&kbar[static_cast<size_t>(i * P.d)]), i);
+  if (P.prefix) {
+    // prefix mean of the own block: keys cB .. p of the query's kv head
+    const int64_t start = kt - p;
+    std::vector<double> pm(static_cast<size_t>(P.d), 0.0);
+    for (int64_t j = c * P.B; j <= p; ++j)
+      for (int x = 0; x < P.d; ++x) pm[x] += load(P.k, P.dtype, kv_off(P, start + j, g) + x);
+    for (int x = 0; x < P.d; ++x) pm[x] /= static_cast<double>(p - c * P.B + 1);
+    s.emplace_back(score(pm.data()), c);
   }
   // Highest score first; equal scores: lower block index first.
   std::sort(s.begin(), s.end(), [](const std::pair<double, int64_t>& a,
@@ -152,14 +181,15 @@ void select_blocks(const Problem& P, int64_t t, int h, int64_t p, const std::vec
     if (a.first != b2.first) return a.first > b2.first;
     return a.second < b2.second;
   });
-  const int64_t nh = std::min<int64_t>(P.topk - 1, c);
+  const int64_t n_cand = static_cast<int64_t>(s.size());
+  const int64_t nh = std::min<int64_t>(P.prefix ? P.topk : P.topk - 1, n_cand);
   std::vector<int32_t> chosen;
   for (int64_t r = 0; r < nh; ++r) chosen.push_back(static_cast<int32_t>(s[r].second));
+  if (!P.prefix) chosen.push_back(static_cast<int32_t>(c));
   std::sort(chosen.begin(), chosen.end());
-  chosen.push_back(static_cast<int32_t>(c));
   for (int r = 0; r < P.topk; ++r) sel[r] = r < static_cast<int>(chosen.size()) ? chosen[r] : -1;
   if (gap) {
-    if (nh > 0 && nh < c) {
+    if (nh > 0 && nh < n_cand) {
       const double a = s[nh - 1].first, b2 = s[nh].first;
       const double den = std::max(std::max(std::fabs(a), std::fabs(b2)), 1e-30);
       *gap = std::fabs(a - b2) / den;
@@ -169,10 +199,20 @@ void select_blocks(const Problem& P, int64_t t, int h, int64_t p, const std::vec
   }
 }
 
+// Whether the query reads its own block: always when it is forced, and with
+// the prefix-mean gate only when the index row names it.
+bool reads_own(const Problem& P, const int32_t* sel, int64_t c) {
+  if (!P.prefix) return true;
+  for (int r = 0; r < P.topk; ++r)
+    if (sel[r] == c) return true;
+  return false;
+}
+
 // Exact softmax attention of query (t, h) over the candidate keys of the
 // chosen blocks: [PT §1 eq.4] with the current block causal [PT §2 eq.5].
 // Entries of sel that are not in [0, c) are not history blocks; block c is
-// always attended up to position p. Returns the number of keys attended.
+// attended up to position p (with P.prefix only if sel names it). Returns the
+// number of keys attended.
 // The query vector is read from Pq at (tq, hq): P itself, or a one-row view
 // of the sampled q rows (oracle_forward_rows with q_rows).
 int64_t attend_q(const Problem& P, const Problem& Pq, int b, int64_t t, int h, int64_t tq, int hq,
@@ -190,7 +230,8 @@ int64_t attend_q(const Problem& P, const Problem& Pq, int b, int64_t t, int h, i
   for (int32_t i : hist)
     for (int64_t j = static_cast<int64_t>(i) * P.B; j < static_cast<int64_t>(i + 1) * P.B; ++j)
       J.push_back(j);
-  for (int64_t j = c * P.B; j <= p; ++j) J.push_back(j);
+  if (reads_own(P, sel, c))
+    for (int64_t j = c * P.B; j <= p; ++j) J.push_back(j);
 
   std::vector<double> logit(J.size());
   double m = -std::numeric_limits<double>::infinity();
@@ -231,7 +272,8 @@ void backward_row(const Problem& P, const void* dout, int b, int64_t t, int h, i
   for (int32_t i : hist)
     for (int64_t j = static_cast<int64_t>(i) * P.B; j < static_cast<int64_t>(i + 1) * P.B; ++j)
       J.push_back(j);
-  for (int64_t j = c * P.B; j <= p; ++j) J.push_back(j);
+  if (reads_own(P, sel, c))
+    for (int64_t j = c * P.B; j <= p; ++j) J.push_back(j);
   const int d = P.d;
   std::vector<double> qv(d), dov(d);
   for (int x = 0; x < d; ++x) {
@@ -311,8 +353,8 @@ int oracle_meanpool(const void* k, int dtype, const int32_t* cu, int batch, int 
 int oracle_gate_topk_routed(const void* q, const void* k, int dtype, const int32_t* cu, int batch,
                             int Hq, int Hkv, int d, int B, int topk, int routing, int32_t* idx,
                             double* gap) {
-  Problem P{q, k, nullptr, dtype, cu, batch, Hq, Hkv, d, B, topk, routing};
-  if (routing != 0 && routing != 1) return -1;
+  Problem P{q, k, nullptr, dtype, cu, batch, Hq, Hkv, d, B, topk, routing & 1, routing >> 1};
+  if (!routing_ok(routing)) return -1;
   if (check(P)) return -1;
   for (int b = 0; b < batch; ++b)
     for (int g = 0; g < Hkv; ++g) {
@@ -325,7 +367,8 @@ int oracle_gate_topk_routed(const void* q, const void* k, int dtype, const int32
         for (int hh = 0; hh < grp; ++hh) {
           const int h = g * grp + hh;
           const int64_t t = cu[b] + p;
-          select_blocks(P, t, h, p, kb, idx + (t * Hq + h) * topk, gap ? gap + t * Hq + h : nullptr);
+          select_blocks(P, t, h, p, kb, idx + (t * Hq + h) * topk, gap ? gap + t * Hq + h : nullptr,
+                        t, g);
         }
     }
   return 0;
@@ -338,8 +381,8 @@ int oracle_forward_routed(const void* q, const void* k, const void* v, int dtype
                           const int32_t* cu, int batch, int Hq, int Hkv, int d, int B, int topk,
                           int routing, const int32_t* idx_in, double* out, double* lse,
                           int32_t* idx_out, int64_t* nkeys) {
-  Problem P{q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk, routing};
-  if (routing != 0 && routing != 1) return -1;
+  Problem P{q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk, routing & 1, routing >> 1};
+  if (!routing_ok(routing)) return -1;
   if (check(P)) return -1;
   for (int b = 0; b < batch; ++b)
     for (int g = 0; g < Hkv; ++g) {
@@ -356,7 +399,7 @@ int oracle_forward_routed(const void* q, const void* k, const void* v, int dtype
           if (idx_in)
             std::memcpy(sel.data(), idx_in + (t * Hq + h) * topk, sizeof(int32_t) * topk);
           else
-            select_blocks(P, t, h, p, kb, sel.data(), nullptr);
+            select_blocks(P, t, h, p, kb, sel.data(), nullptr, t, g);
           if (idx_out) std::memcpy(idx_out + (t * Hq + h) * topk, sel.data(), sizeof(int32_t) * topk);
           const int64_t n = attend(P, b, t, h, p, sel.data(), out + (t * Hq + h) * d,
                                    lse ? lse + t * Hq + h : nullptr);
@@ -375,9 +418,9 @@ int oracle_forward_rows_routed(const void* q, const void* k, const void* v, int 
                                int topk, int routing, const int64_t* rows, int64_t nrows,
                                const int32_t* idx_in, double* out, double* lse, int32_t* idx_out,
                                double* gap, const void* q_rows) {
-  Problem P{q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk, routing};
+  Problem P{q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk, routing & 1, routing >> 1};
   // shared routing reads every head of the group: not with sampled q rows
-  if ((routing != 0 && routing != 1) || (routing == 1 && q_rows)) return -1;
+  if (!routing_ok(routing) || ((routing & 1) && q_rows)) return -1;
   if (check(P)) return -1;
   const int64_t T = batch > 0 ? cu[batch] : 0;
   for (int64_t r = 0; r < nrows; ++r)
@@ -419,7 +462,7 @@ int oracle_forward_rows_routed(const void* q, const void* k, const void* v, int 
       std::memcpy(sel.data(), idx_in + r * topk, sizeof(int32_t) * topk);
     else
       select_blocks(Pr, tq, hq, p, means[static_cast<size_t>(b) * Hkv + h / grp], sel.data(),
-                      &gp);
+                    &gp, t, h / grp);
     if (idx_out) std::memcpy(idx_out + r * topk, sel.data(), sizeof(int32_t) * topk);
     if (gap) gap[r] = gp;
     attend_q(P, Pr, b, t, h, tq, hq, p, sel.data(), out + r * d, lse ? lse + r : nullptr);
@@ -453,8 +496,8 @@ int oracle_backward_routed(const void* q, const void* k, const void* v, const vo
                            const int32_t* cu, int batch, int Hq, int Hkv, int d, int B, int topk,
                            int routing, const int32_t* idx_in, double* dq, double* dk,
                            double* dv) {
-  Problem P{q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk, routing};
-  if (check(P) || (routing != 0 && routing != 1) || !dout) return -1;
+  Problem P{q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk, routing & 1, routing >> 1};
+  if (check(P) || !routing_ok(routing) || !dout) return -1;
   const int64_t T = batch > 0 ? cu[batch] : 0;
   std::fill(dk, dk + T * Hkv * d, 0.0);
   std::fill(dv, dv + T * Hkv * d, 0.0);
@@ -475,7 +518,7 @@ int oracle_backward_routed(const void* q, const void* k, const void* v, const vo
         if (idx_in)
           std::memcpy(sel.data(), idx_in + (t * Hq + h) * topk, sizeof(int32_t) * topk);
         else
-          select_blocks(P, t, h, p, kb, sel.data(), nullptr);
+          select_blocks(P, t, h, p, kb, sel.data(), nullptr, t, g);
         backward_row(P, dout, b, t, h, p, sel.data(), dq, dk, dv);
       }
   }
@@ -485,11 +528,13 @@ int oracle_backward_routed(const void* q, const void* k, const void* v, const vo
 // moba_naive view: per (sequence, head) build the dense boolean mask
 // M[p][j] = (j <= p) and (block(j) is chosen for p), then run dense masked
 // softmax row by row. Uses the gate's choice (or idx_in). [RD], [PT §3.1]
-int oracle_forward_mask(const void* q, const void* k, const void* v, int dtype, const int32_t* cu,
-                        int batch, int Hq, int Hkv, int d, int B, int topk, const int32_t* idx_in,
-                        double* out) {
-  Problem P{q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk};
-  if (check(P)) return -1;
+// With the prefix-mean gate (routing bit 1) the own block is on only when
+// the row names it.
+int oracle_forward_mask_routed(const void* q, const void* k, const void* v, int dtype,
+                               const int32_t* cu, int batch, int Hq, int Hkv, int d, int B,
+                               int topk, int routing, const int32_t* idx_in, double* out) {
+  Problem P{q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk, routing & 1, routing >> 1};
+  if (check(P) || !routing_ok(routing)) return -1;
   const int grp = Hq / Hkv;
   const double scale = 1.0 / std::sqrt(static_cast<double>(d));
   for (int b = 0; b < batch; ++b) {
@@ -507,11 +552,11 @@ int oracle_forward_mask(const void* q, const void* k, const void* v, int dtype, 
         if (idx_in)
           std::memcpy(sel.data(), idx_in + (t * Hq + h) * topk, sizeof(int32_t) * topk);
         else
-          select_blocks(P, t, h, p, kb, sel.data(), nullptr);
+          select_blocks(P, t, h, p, kb, sel.data(), nullptr, t, g);
         const int64_t c = p / B;
         for (int64_t j = 0; j <= p; ++j) {
           const int64_t bj = j / B;
-          bool on = (bj == c);
+          bool on = (bj == c) && !P.prefix;
           for (int r = 0; r < topk && !on; ++r) on = (sel[r] == bj);
           mask[static_cast<size_t>(p * len + j)] = on ? 1 : 0;
         }
@@ -544,6 +589,12 @@ int oracle_forward_mask(const void* q, const void* k, const void* v, int dtype, 
   return 0;
 }
 
+int oracle_forward_mask(const void* q, const void* k, const void* v, int dtype, const int32_t* cu,
+                        int batch, int Hq, int Hkv, int d, int B, int topk, const int32_t* idx_in,
+                        double* out) {
+  return oracle_forward_mask_routed(q, k, v, dtype, cu, batch, Hq, Hkv, d, B, topk, 0, idx_in, out);
+}
+
 // Two-branch route: current block (causal, [PT §2 eq.5]) and history blocks
 // (non-causal, eq.6) each keep (m, l, u); they are merged by eq.(7)-(8).
 // With naive_sum != 0 it instead adds the two separately normalised outputs,
@@ -568,7 +619,7 @@ int oracle_forward_two_branch(const void* q, const void* k, const void* v, int d
           const int64_t t = start + p;
           const int64_t c = p / B;
           std::vector<int32_t> sel(static_cast<size_t>(topk));
-          select_blocks(P, t, h, p, kb, sel.data(), nullptr);
+          select_blocks(P, t, h, p, kb, sel.data(), nullptr, t, g);
           // Branch statistics: m (max logit), l (sum of exp), u (unnormalised sum).
           auto branch = [&](const std::vector<int64_t>& J, double& m, double& l,
                             std::vector<double>& u) {
