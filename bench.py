@@ -2,6 +2,7 @@
 """Benchmark of the B200 MoBA prefill forward pass (one layer-forward = one step).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--variant forced|shared|prefix] [--pass forward|backward]
 
 A step runs the whole path -- block mean-pool, gate/top-k, regrouping,
 history and own-block attention, merge -- on seeded synthetic inputs of the
@@ -17,6 +18,14 @@ slowest rank's time. Prints one JSON line on rank 0.
 
 --impl reference times the fp64 CPU oracle (the only reference this method
 has) on a bounded sample of the same workload on the host cores.
+
+--variant picks the gate: forced own block (default, the headline), shared
+(one choice per kv head's group, by the group's mean score) or prefix (the
+own block scored by the mean of its keys up to the query). Useful FLOPs of
+the prefix variant are counted from the gate's own index rows. --pass
+backward times moba_backward (dq, dk, dv through the chosen blocks, on the
+forward's indices): useful FLOPs 2.5x the forward's (five contractions per
+query-key pair against two).
 """
 from __future__ import annotations
 
@@ -58,6 +67,22 @@ def flop_counts(w):
         dense += int((4 * d * (p + 1)).sum()) * H
     useful = hist + cur
     return useful, hist, cur, dense
+
+
+def flops_from_indices(idx, cu, B, d):
+    """(history, own-block) useful FLOPs of index rows idx [T, Hq, k] (device
+    tensor): every chosen earlier block gives B keys, the own block, when
+    chosen, keys cB..p."""
+    T = idx.shape[0]
+    cu64 = cu.to(idx.device, torch.int64)
+    t = torch.arange(T, device=idx.device)
+    b = torch.searchsorted(cu64[1:], t, right=True)
+    p = t - cu64[b]
+    c = (p // B)[:, None, None]
+    hist = ((idx >= 0) & (idx < c)).sum().item() * B
+    own = (idx == c).any(dim=2)  # [T, Hq]
+    own_keys = ((p - (p // B) * B + 1)[:, None] * own).sum().item()
+    return 4 * d * int(hist), 4 * d * int(own_keys)
 
 
 def row_flops(w, rows):
@@ -200,6 +225,124 @@ def time_oracle(w, q, k, v, cu, budget_s: float, seed: int = 7):
 
 
 # ------------------------------------------------------------ main
+def bench_backward(args, w, moba, q, k, v, cu, dev, world, rank, config, shared, prefix):
+    """--pass backward: moba_backward on the forward's output, lse and index rows."""
+    cu_d = cu.to(dev)
+    out, lse = moba.moba_forward(q, k, v, cu_d, w.block_size, w.topk, max_seqlen=w.max_seqlen,
+                                 return_lse=True, shared_routing=shared, prefix_mean=prefix)
+    idx = moba.moba_gate_topk(q, k, cu_d, w.block_size, w.topk, max_seqlen=w.max_seqlen,
+                              shared_routing=shared, prefix_mean=prefix)
+    gen = torch.Generator(device=dev).manual_seed(w.seed + 17)
+    dout = (torch.randn(q.shape, generator=gen, device=dev) * 0.5).to(q.dtype)
+    if prefix:
+        hist, cur = flops_from_indices(idx, cu, w.block_size, w.head_dim)
+    else:
+        _, hist, cur, _ = flop_counts(w)
+    useful = 2.5 * (hist + cur)
+    p = moba.make_params(q, k, cu, w.block_size, w.topk, w.max_seqlen, shared, prefix)
+    L = moba.lib()
+    P = ctypes.byref(p)
+    L.moba_backward_workspace_size.argtypes = [ctypes.POINTER(moba.MobaParams), ctypes.c_int]
+    L.moba_backward_workspace_size.restype = ctypes.c_size_t
+    fn = L.moba_backward
+    fn.argtypes = [ctypes.POINTER(moba.MobaParams)] + [ctypes.c_void_p] * 12 + [ctypes.c_size_t,
+                                                                              ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    ws = torch.empty(max(int(L.moba_backward_workspace_size(P, 1)), 256), dtype=torch.uint8,
+                     device=dev)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    ptr = lambda x: ctypes.c_void_p(x.data_ptr())
+
+    def step(qq=q, kk=k, vv=v, oo=out, ll=lse, dd=dout, ii=idx):
+        rc = fn(P, ptr(qq), ptr(kk), ptr(vv), ptr(cu_d), ptr(oo), ptr(ll), ptr(dd), ptr(ii),
+                ptr(dq), ptr(dk), ptr(dv), ptr(ws), ws.numel(), sp)
+        if rc:
+            raise RuntimeError(f"moba_backward failed: {rc}")
+
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    if clocks:
+        clocks.wait_first_sample()
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    if moba.moba_device_status(dev) != 0:
+        raise RuntimeError("device status error after warm-up")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t_lo = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_hi = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    if clocks:
+        clocks.stop()
+    clock_info = clocks.summarise(t_lo, t_hi) if clocks else None
+    ms = reduce_max(e0.elapsed_time(e1) / args.steps, world, dev)
+
+    # end to end: the step's inputs from pinned host memory, the gradients back
+    host_in = [x.cpu().pin_memory() for x in (q, k, v, out, lse, dout, idx)]
+    dev_in = [torch.empty_like(x) for x in (q, k, v, out, lse, dout, idx)]
+    host_out = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in (dq, dk, dv)]
+
+    def e2e_step():
+        for d_, h_ in zip(dev_in, host_in):
+            d_.copy_(h_, non_blocking=True)
+        step(*dev_in)
+        for h_, d_ in zip(host_out, (dq, dk, dv)):
+            h_.copy_(d_, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    erep = max(3, min(args.steps, 10))
+    e0.record(stream)
+    for _ in range(erep):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / erep, world, dev)
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    value = useful * world / (ms * 1e-3) / 1e12
+    line = {
+        "metric": "moba_prefill_bwd_useful_tflops", "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": dict(config, **{"pass": "backward"}),
+        "roofline": {"bound": "tensor", "achieved": value / world, "peak": peak,
+                     "unit": "TFLOP/s", "frac": value / world / peak, "traffic": None,
+                     "kernel": "moba_backward, all launches (a lower bound for each kernel)",
+                     "peak_source": f"{peak_src} bf16 burst"},
+        "cpu_baseline": None,
+        "e2e": {"value": useful * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in host_in),
+                "d2h_bytes_per_step": sum(x.numel() * x.element_size() for x in host_out)},
+        # regroup (4), D = dO . O, the history and own-block kernels
+        "gpu_launches": 7 * args.steps,
+        "clocks": clock_info,
+        "useful_flop_per_step": useful,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -209,6 +352,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--variant", default="forced", choices=["forced", "shared", "prefix"])
+    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"])
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -219,6 +364,8 @@ def main():
               "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
               "block_size": w.block_size, "topk": w.topk,
               "l2": "inputs exceed L2 (q+k+v > 126 MB), no flush"}
+    if args.variant != "forced":
+        config["variant"] = args.variant
     dtype_name = "bf16" if w.dtype == torch.bfloat16 else "f32"
 
     if args.impl == "reference":
@@ -257,8 +404,17 @@ def main():
     torch.cuda.set_device(dev)
     q, k, v, cu = make_inputs(rank_workload(w, rank), dev)
     cu_d = cu.to(dev)
-    p = moba.make_params(q, k, cu, w.block_size, w.topk, w.max_seqlen)
+    shared, prefix = args.variant == "shared", args.variant == "prefix"
+    if args.pass_ == "backward":
+        return bench_backward(args, w, moba, q, k, v, cu, dev, world, rank, config, shared, prefix)
+    p = moba.make_params(q, k, cu, w.block_size, w.topk, w.max_seqlen, shared, prefix)
     ws = moba.workspace(p, dev)
+    if prefix:
+        idx0 = moba.moba_gate_topk(q, k, cu_d, w.block_size, w.topk, max_seqlen=w.max_seqlen,
+                                   prefix_mean=True)
+        hist_flops, cur_flops = flops_from_indices(idx0, cu, w.block_size, w.head_dim)
+        useful = hist_flops + cur_flops
+        del idx0
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream(dev)
     L = moba.lib()
@@ -393,13 +549,15 @@ def main():
     tc_path = w.dtype == torch.bfloat16 and w.head_dim == 128 and w.block_size % 128 == 0
     # mean-pool, gate; per pass: 4 regroup kernels, history, own-block (+ merge on the SIMT path)
     launches_per_step = 2 + (6 if tc_path else 7) * n_pass
+    if prefix:  # the own-block scores: chunk key sums, then the dot products
+        launches_per_step += 2
 
     if rank != 0:
         if world > 1:
             torch.distributed.destroy_process_group()
         return
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and args.variant == "forced":
         tf, nrows, dt, thr = time_oracle(w, q, k, v, cu, args.cpu_budget)
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                "sample": f"{nrows} seeded (token, head) rows of {w.name} ({dt:.1f} s), "

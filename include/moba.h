@@ -19,7 +19,7 @@
  *   Blocks restart at every sequence start (block i of sequence b covers its
  *   positions iB .. iB+B-1); no key crosses a sequence boundary.
  * Heads: q head h reads kv head h / (Hq / Hkv) (grouped-query attention);
- *   routing is done per q head.
+ *   routing is done per q head (moba_params.routing, .own_block: variants).
  * Element type: bf16 or fp32 (moba_params.dtype) for q, k, v and out;
  *   arithmetic is fp32 (bf16 tensor-core products, fp32 accumulation).
  * Pointers: every data pointer is a DEVICE pointer owned by the caller,
@@ -74,9 +74,19 @@ typedef struct {
   int routing;       /* 0 (default): every query head chooses its own blocks.
                         1: the query heads of a kv head's group share one choice,
                         made on the group's mean score (1/grp) sum_h q_h . kbar_i
-                        (PaperTrace "2.1.3 MoBA", section 5.4, multi-head
+                        (PaperTrace "2.1.3 MoBA", section 5.5, multi-head
                         settings: a group sharing candidates must aggregate its
                         heads' scores; the mean is this library's reading). */
+  int own_block;     /* 0 (default): the query's own block c is always chosen and
+                        takes one of the k slots. 1: block c is scored by the
+                        mean of its keys up to and including the query (the
+                        prefix mean, PaperTrace "2.1.3 MoBA", section 5.2 on
+                        causal blocks) and competes with blocks 0..c-1; the k
+                        slots go to the best min(k, c+1) blocks, ties to the
+                        lower index. A query whose own block loses reads no key
+                        of it, itself included; its index row then lists only
+                        earlier blocks. With routing 1 the group's mean of the
+                        own-block scores is used. */
 } moba_params;
 
 /* Number of key blocks reserved per sequence: ceil(max_seqlen / B). */
@@ -100,7 +110,10 @@ MOBA_API moba_status moba_meanpool(const moba_params* p, const void* k, const in
  * ascending order -- the chosen earlier blocks first, then the query's own
  * block c -- padded with -1 to k entries. Only blocks i < c are scored
  * (s_i = q . kbar_i, fp32); blocks after c are never chosen; ties go to the
- * lower block index. idx: int32 [T][Hq][k]. Uses the workspace for kbar. */
+ * lower block index. idx: int32 [T][Hq][k]. With own_block = 1 the own
+ * block is a scored candidate (prefix mean) and appears only if chosen.
+ * Uses the workspace for kbar (and, with own_block = 1, for the own-block
+ * scores: T * Hq floats). */
 MOBA_API moba_status moba_gate_topk(const moba_params* p, const void* q, const void* k,
                            const int32_t* cu_seqlens, int32_t* idx, void* ws, size_t ws_bytes,
                            void* stream);
@@ -120,7 +133,8 @@ MOBA_API moba_status moba_gate_topk(const moba_params* p, const void* q, const v
  * All calls share the one array and it keeps the last call's contents
  * (nothing in it has to start at zero); calls that overlap on the GPU --
  * on different streams, or from different host threads -- race on it.
- * Device-side checks of cu_seqlens are not recorded in the status word. */
+ * Device-side checks of cu_seqlens are not recorded in the status word.
+ * own_block = 1 needs workspace for its scores: MOBA_ERR_UNSUPPORTED. */
 MOBA_API moba_status moba_gate_topk_noalloc(const moba_params* p, const void* q, const void* k,
                                             const int32_t* cu_seqlens, int32_t* idx,
                                             void* stream);
@@ -155,7 +169,8 @@ MOBA_API moba_status moba_forward_staged(const moba_params* p, const void* q, co
  * the gate (forced candidates; a sliding-window or sink pattern is a special
  * gate, section 3). idx: int32 [T][Hq][k] in the canonical form that
  * moba_gate_topk writes: strictly ascending earlier blocks (each < c), then
- * c, then -1. A row not in that form records MOBA_ERR_BAD_INDICES in the
+ * c, then -1 (with own_block = 1, c may be absent: the row then reads no
+ * key of the own block). A row not in that form records MOBA_ERR_BAD_INDICES in the
  * device status word; its output is then unspecified, but every access stays
  * in bounds. */
 MOBA_API moba_status moba_forward_with_indices(const moba_params* p, const void* q, const void* k,

@@ -33,7 +33,7 @@ class MobaParams(ctypes.Structure):
                 ("max_seqlen", ctypes.c_int), ("num_q_heads", ctypes.c_int),
                 ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
                 ("block_size", ctypes.c_int), ("topk", ctypes.c_int), ("dtype", ctypes.c_int),
-                ("routing", ctypes.c_int)]
+                ("routing", ctypes.c_int), ("own_block", ctypes.c_int)]
 
 
 class MobaError(RuntimeError):
@@ -80,7 +80,7 @@ def _check(fn: str, code: int) -> None:
 
 def make_params(q: torch.Tensor, k: torch.Tensor, cu_seqlens: torch.Tensor, block_size: int,
                 topk: int, max_seqlen: Optional[int] = None,
-                shared_routing: bool = False) -> MobaParams:
+                shared_routing: bool = False, prefix_mean: bool = False) -> MobaParams:
     T, Hq, d = q.shape
     Hkv = k.shape[1]
     batch = cu_seqlens.numel() - 1
@@ -94,7 +94,7 @@ def make_params(q: torch.Tensor, k: torch.Tensor, cu_seqlens: torch.Tensor, bloc
     else:
         raise TypeError(f"unsupported dtype {q.dtype}")
     return MobaParams(batch, T, max_seqlen, Hq, Hkv, d, block_size, topk, dt,
-                      1 if shared_routing else 0)
+                      1 if shared_routing else 0, 1 if prefix_mean else 0)
 
 
 def _ptr(x: Optional[torch.Tensor]):
@@ -142,11 +142,14 @@ def moba_meanpool(k: torch.Tensor, cu_seqlens: torch.Tensor, block_size: int,
 
 
 def moba_gate_topk(q, k, cu_seqlens, block_size: int, topk: int, max_seqlen=None,
-                   ws: Optional[torch.Tensor] = None, shared_routing: bool = False) -> torch.Tensor:
+                   ws: Optional[torch.Tensor] = None, shared_routing: bool = False,
+                   prefix_mean: bool = False) -> torch.Tensor:
     """Chosen blocks per (token, q head): int32 [T, Hq, topk], ascending, -1 padded.
-    shared_routing: the q heads of a kv head's group share the blocks of their mean score."""
+    shared_routing: the q heads of a kv head's group share the blocks of their mean score.
+    prefix_mean: the own block is scored by the mean of its keys up to the query and competes
+    for the k slots instead of being forced."""
     _check_inputs(q, k)
-    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen, shared_routing)
+    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen, shared_routing, prefix_mean)
     cu = _dev_i32(cu_seqlens, q.device)
     ws = workspace(p, q.device) if ws is None else ws
     idx = torch.empty((p.total_tokens, p.num_q_heads, topk), dtype=torch.int32, device=q.device)
@@ -179,11 +182,14 @@ def moba_gate_topk_noalloc(q, k, cu_seqlens, block_size: int, topk: int, max_seq
 
 def moba_forward(q, k, v, cu_seqlens, block_size: int, topk: int, max_seqlen=None,
                  return_lse: bool = False, ws: Optional[torch.Tensor] = None,
-                 out: Optional[torch.Tensor] = None, shared_routing: bool = False):
+                 out: Optional[torch.Tensor] = None, shared_routing: bool = False,
+                 prefix_mean: bool = False):
     """MoBA prefill forward: out [T, Hq, d] (input dtype) and optionally lse [T, Hq].
-    shared_routing: the q heads of a kv head's group share the blocks of their mean score."""
+    shared_routing: the q heads of a kv head's group share the blocks of their mean score.
+    prefix_mean: the own block is scored by the mean of its keys up to the query and competes
+    for the k slots instead of being forced."""
     _check_inputs(q, k, v)
-    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen, shared_routing)
+    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen, shared_routing, prefix_mean)
     cu = _dev_i32(cu_seqlens, q.device)
     ws = workspace(p, q.device) if ws is None else ws
     out = torch.empty_like(q) if out is None else out
@@ -196,13 +202,13 @@ def moba_forward(q, k, v, cu_seqlens, block_size: int, topk: int, max_seqlen=Non
 
 def moba_backward(q, k, v, cu_seqlens, out, lse, dout, block_size: int, topk: int,
                   idx: Optional[torch.Tensor] = None, max_seqlen=None,
-                  shared_routing: bool = False):
+                  shared_routing: bool = False, prefix_mean: bool = False):
     """Gradients of sum(dout * out) through the chosen blocks: (dq [T,Hq,d], dk, dv [T,Hkv,d])
     in fp32. out, lse: the forward's results; idx: its index rows, or None to run the gate
     again."""
     _check_inputs(q, k, v, out, dout, lse, idx)
     L = lib()
-    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen, shared_routing)
+    p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen, shared_routing, prefix_mean)
     cu = _dev_i32(cu_seqlens, q.device)
     L.moba_backward_workspace_size.argtypes = [ctypes.POINTER(MobaParams), ctypes.c_int]
     L.moba_backward_workspace_size.restype = ctypes.c_size_t
@@ -222,10 +228,12 @@ def moba_backward(q, k, v, cu_seqlens, out, lse, dout, block_size: int, topk: in
 
 
 def moba_forward_with_indices(q, k, v, cu_seqlens, idx, block_size: int, max_seqlen=None,
-                              return_lse: bool = False, ws: Optional[torch.Tensor] = None):
-    """MoBA forward with caller-chosen blocks idx int32 [T, Hq, topk] (canonical form)."""
+                              return_lse: bool = False, ws: Optional[torch.Tensor] = None,
+                              prefix_mean: bool = False):
+    """MoBA forward with caller-chosen blocks idx int32 [T, Hq, topk] (canonical form; with
+    prefix_mean a row may leave out its own block and then reads none of it)."""
     _check_inputs(q, k, v, idx)
-    p = make_params(q, k, cu_seqlens, block_size, idx.shape[2], max_seqlen)
+    p = make_params(q, k, cu_seqlens, block_size, idx.shape[2], max_seqlen, prefix_mean=prefix_mean)
     cu = _dev_i32(cu_seqlens, q.device)
     ws = workspace(p, q.device) if ws is None else ws
     out = torch.empty_like(q)

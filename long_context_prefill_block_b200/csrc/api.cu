@@ -44,6 +44,7 @@ moba_status validate(const moba_params* p, Dims& dm) {
       p->topk <= 0)
     return MOBA_ERR_INVALID_ARG;
   if (p->routing != 0 && p->routing != 1) return MOBA_ERR_INVALID_ARG;
+  if (p->own_block != 0 && p->own_block != 1) return MOBA_ERR_INVALID_ARG;
   if (p->dtype != MOBA_BF16 && p->dtype != MOBA_F32) return MOBA_ERR_UNSUPPORTED;
   if (p->head_dim != 64 && p->head_dim != 128) return MOBA_ERR_UNSUPPORTED;
   if (p->topk > 32) return MOBA_ERR_UNSUPPORTED;
@@ -61,16 +62,40 @@ moba_status validate(const moba_params* p, Dims& dm) {
   dm.nb = (int)(((int64_t)p->max_seqlen + p->block_size - 1) / p->block_size);
   dm.dtype = p->dtype == MOBA_BF16 ? kBF16 : kF32;
   dm.shared = p->routing;
+  dm.prefix = p->own_block;
   return MOBA_OK;
 }
 
 bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; }
 
 struct Layout {
-  size_t kbar, idx, counts, cursor, list_off, tile_off, pairs, tiles, part_o, part_lse, total;
+  size_t kbar, own, idx, counts, cursor, list_off, tile_off, pairs, tiles, part_o, part_lse, total;
   int ng;             // kv heads per pass
   int64_t max_tiles;  // tile-table capacity per pass
 };
+
+// Own-block scores of the prefix-mean gate, when the gate runs: fp32 [T][Hq],
+// then the per-chunk key sums they are built from.
+size_t own_scores_bytes(const Dims& dm) { return (sizeof(float) * (size_t)dm.T * dm.Hq + 255) & ~size_t(255); }
+size_t own_score_bytes(const Dims& dm, bool gate_runs) {
+  if (!dm.prefix || !gate_runs) return 0;
+  return own_scores_bytes(dm) + sizeof(float) * (size_t)dm.batch * dm.nb *
+                                    own_chunks_per_block(dm) * dm.Hkv * dm.d;
+}
+float* own_chunk_sums(float* own, const Dims& dm) {
+  return reinterpret_cast<float*>(reinterpret_cast<char*>(own) + own_scores_bytes(dm));
+}
+
+// Runs the gate: block means, the own-block scores of the prefix-mean
+// variant, then gate/top-k.
+cudaError_t run_gate(const Dims& dm, const void* q, const void* k, const int32_t* cu, float* kbar,
+                     float* own, int32_t* idx, int* status, cudaStream_t st) {
+  cudaError_t e = launch_meanpool(dm, k, cu, kbar, status, st);
+  if (e == cudaSuccess && dm.prefix)
+    e = launch_own_score(dm, q, k, cu, own, own_chunk_sums(own, dm), status, st);
+  if (e == cudaSuccess) e = launch_gate(dm, q, kbar, own, cu, idx, status, st);
+  return e;
+}
 
 // Workspace plan. `own_idx` reserves room for the index rows (moba_forward).
 Layout plan(const Dims& dm, bool own_idx) {
@@ -82,7 +107,7 @@ Layout plan(const Dims& dm, bool own_idx) {
   if (ng > (size_t)dm.Hkv) ng = dm.Hkv;
   L.ng = (int)ng;
   const int64_t n_lists = (int64_t)dm.batch * L.ng * dm.nb;
-  const int64_t max_pairs = (int64_t)dm.T * L.ng * grp * (dm.topk - 1);
+  const int64_t max_pairs = (int64_t)dm.T * L.ng * grp * hist_slots(dm);
   const int tile_m = kSimtTileM < tc_tile_m() ? kSimtTileM : tc_tile_m();
   L.max_tiles = (max_pairs + tile_m - 1) / tile_m + n_lists;
   size_t off = 0;
@@ -92,6 +117,7 @@ Layout plan(const Dims& dm, bool own_idx) {
     return at;
   };
   L.kbar = take(sizeof(float) * (size_t)dm.batch * dm.nb * dm.Hkv * dm.d);
+  L.own = take(own_score_bytes(dm, own_idx));
   L.idx = take(own_idx ? sizeof(int32_t) * (size_t)dm.T * dm.Hq * dm.topk : 0);
   L.counts = take(sizeof(int32_t) * n_lists);
   L.cursor = take(sizeof(int32_t) * n_lists);
@@ -157,7 +183,10 @@ moba_status forward_impl(const moba_params* p, const void* q, const void* k, con
     int32_t* own = reinterpret_cast<int32_t*>(base + L.idx);
     MOBA_TRY(launch_meanpool(dm, k, cu, kbar, status, st));
     MOBA_TRY(mark());
-    MOBA_TRY(launch_gate(dm, q, kbar, cu, own, status, st));
+    float* own_score = reinterpret_cast<float*>(base + L.own);
+    if (dm.prefix)
+      MOBA_TRY(launch_own_score(dm, q, k, cu, own_score, own_chunk_sums(own_score, dm), status, st));
+    MOBA_TRY(launch_gate(dm, q, kbar, own_score, cu, own, status, st));
     MOBA_TRY(mark());
     idx = own;
   } else {
@@ -182,7 +211,7 @@ moba_status forward_impl(const moba_params* p, const void* q, const void* k, con
     ch.nq = ch.ng * grp;
     ch.n_lists = dm.batch * ch.ng * dm.nb;
     ch.tile_m = tc ? tc_tile_m() : kSimtTileM;
-    const int64_t pairs = (int64_t)dm.T * ch.nq * (dm.topk - 1);
+    const int64_t pairs = (int64_t)dm.T * ch.nq * hist_slots(dm);
     rg.max_tiles = (pairs + ch.tile_m - 1) / ch.tile_m + ch.n_lists;
     MOBA_TRY(launch_regroup(dm, ch, idx, cu, rg, status, st));
     MOBA_TRY(mark());
@@ -207,14 +236,14 @@ moba_status forward_impl(const moba_params* p, const void* q, const void* k, con
 // Backward workspace: block means and index rows when the gate runs again,
 // the regroup lists of every kv head (one pass), and D = dO . O per row.
 struct BwdLayout {
-  size_t kbar, idx, counts, cursor, list_off, tile_off, pairs, tiles, dsum, total;
+  size_t kbar, own, idx, counts, cursor, list_off, tile_off, pairs, tiles, dsum, total;
   int64_t max_tiles;
 };
 
 BwdLayout plan_bwd(const Dims& dm, bool own_idx) {
   BwdLayout L{};
   const int64_t n_lists = (int64_t)dm.batch * dm.Hkv * dm.nb;
-  const int64_t max_pairs = (int64_t)dm.T * dm.Hq * (dm.topk - 1);
+  const int64_t max_pairs = (int64_t)dm.T * dm.Hq * hist_slots(dm);
   L.max_tiles = (max_pairs + kSimtTileM - 1) / kSimtTileM + n_lists;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -223,6 +252,7 @@ BwdLayout plan_bwd(const Dims& dm, bool own_idx) {
     return at;
   };
   L.kbar = take(own_idx ? sizeof(float) * (size_t)dm.batch * dm.nb * dm.Hkv * dm.d : 0);
+  L.own = take(own_score_bytes(dm, own_idx));
   L.idx = take(own_idx ? sizeof(int32_t) * (size_t)dm.T * dm.Hq * dm.topk : 0);
   L.counts = take(sizeof(int32_t) * n_lists);
   L.cursor = take(sizeof(int32_t) * n_lists);
@@ -261,8 +291,7 @@ moba_status backward_impl(const moba_params* p, const void* q, const void* k, co
   if (!idx_in) {
     float* kbar = reinterpret_cast<float*>(base + L.kbar);
     int32_t* own = reinterpret_cast<int32_t*>(base + L.idx);
-    MOBA_TRY(launch_meanpool(dm, k, cu, kbar, status, st));
-    MOBA_TRY(launch_gate(dm, q, kbar, cu, own, status, st));
+    MOBA_TRY(run_gate(dm, q, k, cu, kbar, reinterpret_cast<float*>(base + L.own), own, status, st));
     idx = own;
   }
   Regroup rg;
@@ -284,9 +313,10 @@ moba_status backward_impl(const moba_params* p, const void* q, const void* k, co
   float* dsum = reinterpret_cast<float*>(base + L.dsum);
   MOBA_TRY(launch_bwd_dot(dm, out, dout, dsum, st));
   if (bwd_tc_supported(dm))
-    MOBA_TRY(launch_backward_tc(dm, ch, q, k, v, dout, lse, dsum, cu, rg, dq, dk, dv, status, st));
+    MOBA_TRY(launch_backward_tc(dm, ch, q, k, v, dout, lse, dsum, cu, idx, rg, dq, dk, dv, status,
+                                st));
   else
-    MOBA_TRY(launch_backward(dm, ch, q, k, v, dout, lse, dsum, cu, rg, dq, dk, dv, status, st));
+    MOBA_TRY(launch_backward(dm, ch, q, k, v, dout, lse, dsum, cu, idx, rg, dq, dk, dv, status, st));
   return MOBA_OK;
 }
 
@@ -341,16 +371,18 @@ moba_status moba_gate_topk(const moba_params* p, const void* q, const void* k,
   if (s != MOBA_OK) return s;
   if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
   if (!q || !k || !cu_seqlens || !idx || !aligned16(q) || !aligned16(k)) return MOBA_ERR_INVALID_ARG;
+  // the gate needs the block means and, for the prefix-mean variant, the
+  // own-block scores: the head of the forward's workspace plan
   const Layout L = plan(dm, true);
-  if (!ws || ws_bytes < L.kbar + sizeof(float) * (size_t)dm.batch * dm.nb * dm.Hkv * dm.d ||
-      !aligned16(ws))
-    return MOBA_ERR_WORKSPACE;
+  const size_t need = dm.prefix ? L.own + own_score_bytes(dm, true)
+                                : L.kbar + sizeof(float) * (size_t)dm.batch * dm.nb * dm.Hkv * dm.d;
+  if (!ws || ws_bytes < need || !aligned16(ws)) return MOBA_ERR_WORKSPACE;
   int* status = status_word();
   if (!status) return MOBA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* kbar = reinterpret_cast<float*>(static_cast<char*>(ws) + L.kbar);
-  MOBA_TRY(launch_meanpool(dm, k, cu_seqlens, kbar, status, st));
-  MOBA_TRY(launch_gate(dm, q, kbar, cu_seqlens, idx, status, st));
+  char* base = static_cast<char*>(ws);
+  MOBA_TRY(run_gate(dm, q, k, cu_seqlens, reinterpret_cast<float*>(base + L.kbar),
+                    reinterpret_cast<float*>(base + L.own), idx, status, st));
   return MOBA_OK;
 }
 

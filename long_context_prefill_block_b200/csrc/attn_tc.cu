@@ -200,10 +200,14 @@ __device__ __forceinline__ Tile half_view(const Tile& T, int h) {
 
 // Identity of query row r of a tile: the q row it reads (t * Hq + h, or -1)
 // and, for outputs, the token t, head h, position p and partial row prow.
+// Own-block rows (CUR): prow is the row's first partial slot, nhist the
+// number of history partials before the own block's slot, and own whether
+// the row reads its own block (a row whose own block lost the prefix-mean
+// gate merges its history alone).
 struct Row {
-  bool has_q, valid;
+  bool has_q, valid, own;
   int64_t t, prow;
-  int h, p;
+  int h, p, nhist;
 };
 
 template <int MODE>
@@ -227,11 +231,15 @@ __device__ __forceinline__ Row get_row(const Args& a, const Tile& T, int r) {
   if (MODE == CUR && R.valid) {
     const int c = R.p / dm.B;
     const int32_t* row = a.idx + (R.t * dm.Hq + R.h) * (int64_t)dm.topk;
-    int slot = -1;
-    for (int i = 0; i < dm.topk; ++i)
+    int slot = -1, n = 0;
+    for (int i = 0; i < dm.topk; ++i) {
       if (row[i] == c && slot < 0) slot = i;
-    R.prow = (R.t * a.ch.nq + (R.h - a.ch.h0)) * (int64_t)dm.topk + (slot < 0 ? 0 : slot);
-    R.valid = slot >= 0;
+      n += row[i] >= 0 && row[i] < c;
+    }
+    R.prow = (R.t * a.ch.nq + (R.h - a.ch.h0)) * (int64_t)dm.topk;
+    R.own = slot >= 0;
+    R.nhist = R.own ? slot : n;
+    R.valid = R.own || dm.prefix;
   }
   return R;
 }
@@ -591,9 +599,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
         // sum_j w_j) and write the output; the own result never leaves the
         // SM. Slots 0..slot-1 of the row hold the history partials. Each
         // thread merges its own row with 32 independent 16-byte loads per
-        // slot in flight.
-        const int slot = R.valid ? (int)(R.prow % dm.topk) : 0;
-        const int64_t prow0 = R.valid ? R.prow - slot : 0;
+        // slot in flight. A row whose own block lost the prefix-mean gate
+        // gives its own result weight 0.
+        const int slot = R.valid ? R.nhist : 0;
+        const int64_t prow0 = R.valid ? R.prow : 0;
         const int64_t orow = R.valid ? R.t * dm.Hq + R.h : -1;
         float o[D];
 #pragma unroll
@@ -608,9 +617,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
         fence_before_sync();
         mbar_arrive(&sh.o_free[hh]);
         if (R.valid) {
-          float m = lse;
+          float m = R.own ? lse : -INFINITY;
           for (int j = 0; j < slot; ++j) m = fmaxf(m, a.part_lse[prow0 + j]);
-          const float w_own = ex2((lse - m) * 1.4426950408889634f);
+          const float w_own = R.own ? ex2((lse - m) * 1.4426950408889634f) : 0.f;
           float L = w_own;
 #pragma unroll
           for (int x = 0; x < D; ++x) o[x] *= w_own;

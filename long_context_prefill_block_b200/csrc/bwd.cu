@@ -43,6 +43,7 @@ struct BwdArgs {
   const float* lse;   // [T][Hq], natural log
   const float* Dsum;  // [T][Hq], dO . O
   const int32_t* cu;
+  const int32_t* idx;  // [T][Hq][k] index rows (own-block rows of the prefix-mean gate)
   const int32_t* list_off;
   const int32_t* pairs;
   float* dq;  // [T][Hq][d]
@@ -168,7 +169,8 @@ __global__ void __launch_bounds__(kThreads) bwd_block_kernel(const BwdArgs a) {
           const int p = p_first + (int)(i / grp);
           const int h = g * grp + (int)(i % grp);
           qrow = (start + p) * dm.Hq + h;
-          pos = p;
+          // a row whose own block lost the prefix-mean gate reads none of it
+          pos = reads_own(dm, a.idx + qrow * dm.topk, p / dm.B) ? p : -1;
         }
         lse_s[tid] = a.lse[qrow];
         D_s[tid] = a.Dsum[qrow];
@@ -327,8 +329,8 @@ cudaError_t launch_bwd_dot(const Dims& dm, const void* out, const void* dout, fl
 
 cudaError_t launch_backward(const Dims& dm, const Chunk& ch, const void* q, const void* k,
                             const void* v, const void* dout, const float* lse, const float* Dsum,
-                            const int32_t* cu, const Regroup& rg, float* dq, float* dk, float* dv,
-                            int* status, cudaStream_t st) {
+                            const int32_t* cu, const int32_t* idx, const Regroup& rg, float* dq,
+                            float* dk, float* dv, int* status, cudaStream_t st) {
   if (dm.batch == 0 || dm.max_seqlen == 0) return cudaSuccess;
   BwdArgs a{};
   a.dm = dm;
@@ -340,6 +342,7 @@ cudaError_t launch_backward(const Dims& dm, const Chunk& ch, const void* q, cons
   a.lse = lse;
   a.Dsum = Dsum;
   a.cu = cu;
+  a.idx = idx;
   a.list_off = rg.list_off;
   a.pairs = rg.pairs;
   a.dq = dq;

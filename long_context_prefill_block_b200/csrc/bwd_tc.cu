@@ -50,6 +50,7 @@ struct Args {
   const float* lse;
   const float* Dsum;
   const int32_t* cu;
+  const int32_t* idx;  // [T][Hq][k] index rows (own-block rows of the prefix-mean gate)
   const int32_t* list_off;
   const int32_t* pairs;
   float* dq;
@@ -157,7 +158,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ C
       } else {
         const int p = p_first + (int)(i / grp);
         qrow = (start + p) * dm.Hq + g * grp + (int)(i % grp);
-        pos = p;
+        // a row whose own block lost the prefix-mean gate reads none of it
+        pos = reads_own(dm, a.idx + qrow * dm.topk, p / dm.B) ? p : -1;
       }
       lse_r = a.lse[qrow];
       d_r = a.Dsum[qrow];
@@ -352,8 +354,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ C
 
 cudaError_t launch_backward_tc(const Dims& dm, const Chunk& ch, const void* q, const void* k,
                                const void* v, const void* dout, const float* lse,
-                               const float* Dsum, const int32_t* cu, const Regroup& rg,
-                               float* dq, float* dk, float* dv, int* status, cudaStream_t st) {
+                               const float* Dsum, const int32_t* cu, const int32_t* idx,
+                               const Regroup& rg, float* dq, float* dk, float* dv, int* status,
+                               cudaStream_t st) {
   if (dm.batch == 0 || dm.max_seqlen == 0) return cudaSuccess;
   CUtensorMap mk, mv;
   cudaError_t e;
@@ -367,6 +370,7 @@ cudaError_t launch_backward_tc(const Dims& dm, const Chunk& ch, const void* q, c
   a.lse = lse;
   a.Dsum = Dsum;
   a.cu = cu;
+  a.idx = idx;
   a.list_off = rg.list_off;
   a.pairs = rg.pairs;
   a.dq = dq;

@@ -28,7 +28,28 @@ struct Dims {
   int nb;          // blocks reserved per sequence = ceil(max_seqlen / B)
   int dtype;       // kBF16 / kF32
   int shared;      // 1: a kv head's query heads share the blocks of their mean score
+  int prefix;      // 1: the own block is scored by its prefix mean instead of forced
 };
+
+// History slots an index row can hold: k - 1 beside the forced own block,
+// all k when the own block competes for its slot.
+__host__ __device__ inline int hist_slots(const Dims& dm) { return dm.prefix ? dm.topk : dm.topk - 1; }
+
+// The prefix-mean own-block scores are built from per-chunk key sums: a
+// block is split into chunks of kOwnChunkRows rows.
+constexpr int kOwnChunkRows = 32;
+__host__ __device__ inline int own_chunks_per_block(const Dims& dm) {
+  return (dm.B + kOwnChunkRows - 1) / kOwnChunkRows;
+}
+
+// Whether query row `row` (k entries) reads its own block c: always when the
+// own block is forced, else when the row names it.
+__device__ __forceinline__ bool reads_own(const Dims& dm, const int32_t* row, int c) {
+  if (!dm.prefix) return true;
+  bool on = false;
+  for (int r = 0; r < dm.topk; ++r) on |= row[r] == c;
+  return on;
+}
 
 // Work of one pass over a group of kv heads [g0, g0 + ng): its q heads are
 // [g0 * grp, (g0 + ng) * grp). Partial results are indexed by
@@ -103,10 +124,15 @@ cudaError_t launch_meanpool(const Dims& dm, const void* k, const int32_t* cu, fl
                             int* status, cudaStream_t st);
 // Tensor-core gate (bf16, d = 128, at most 256 blocks per sequence).
 bool gate_tc_supported(const Dims& dm);
-cudaError_t launch_gate_tc(const Dims& dm, const void* q, const float* kbar, const int32_t* cu,
-                           int32_t* idx, int* status, cudaStream_t st);
-cudaError_t launch_gate(const Dims& dm, const void* q, const float* kbar, const int32_t* cu,
-                        int32_t* idx, int* status, cudaStream_t st);
+cudaError_t launch_gate_tc(const Dims& dm, const void* q, const float* kbar, const float* own,
+                           const int32_t* cu, int32_t* idx, int* status, cudaStream_t st);
+// own: with dm.prefix, the own-block scores [T][Hq] (launch_own_score); else unused.
+cudaError_t launch_gate(const Dims& dm, const void* q, const float* kbar, const float* own,
+                        const int32_t* cu, int32_t* idx, int* status, cudaStream_t st);
+// Own-block scores by prefix mean: own[t][h] = q_{t,h} . mean(k_{cB..p}) (fp32).
+// csum: scratch for the chunk key sums, batch * nb * own_chunks_per_block * Hkv * d floats.
+cudaError_t launch_own_score(const Dims& dm, const void* q, const void* k, const int32_t* cu,
+                             float* own, float* csum, int* status, cudaStream_t st);
 
 // Regrouping of (query, head, slot) by the history block it chose.
 struct Regroup {
@@ -142,14 +168,15 @@ cudaError_t launch_bwd_dot(const Dims& dm, const void* out, const void* dout, fl
                            cudaStream_t st);
 cudaError_t launch_backward(const Dims& dm, const Chunk& ch, const void* q, const void* k,
                             const void* v, const void* dout, const float* lse, const float* Dsum,
-                            const int32_t* cu, const Regroup& rg, float* dq, float* dk, float* dv,
-                            int* status, cudaStream_t st);
+                            const int32_t* cu, const int32_t* idx, const Regroup& rg, float* dq,
+                            float* dk, float* dv, int* status, cudaStream_t st);
 // Tensor-core backward (bf16, d = 128, B % 128 == 0).
 bool bwd_tc_supported(const Dims& dm);
 cudaError_t launch_backward_tc(const Dims& dm, const Chunk& ch, const void* q, const void* k,
                                const void* v, const void* dout, const float* lse,
-                               const float* Dsum, const int32_t* cu, const Regroup& rg,
-                               float* dq, float* dk, float* dv, int* status, cudaStream_t st);
+                               const float* Dsum, const int32_t* cu, const int32_t* idx,
+                               const Regroup& rg, float* dq, float* dk, float* dv, int* status,
+                               cudaStream_t st);
 constexpr int kSimtTileM = 32;
 
 cudaError_t launch_merge(const Dims& dm, const Chunk& ch, const int32_t* idx, const int32_t* cu,

@@ -14,6 +14,13 @@
 // memory) writes the chunk's scores to shared memory, then 4 threads per
 // query scan them into sorted register lists of their best KM >= k-1
 // blocks; at the end the four lists are merged by warp shuffles.
+//
+// Own-block variant (section 5.2, causal blocks): with dm.prefix the own
+// block c is not forced but scored by its prefix mean (own[t][h], from
+// launch_own_score) and competes for the k slots: the k best of blocks
+// 0..c win, equal scores going to the lower index, so c loses a tie. Block
+// c is in iff fewer than k earlier blocks score at least as high, i.e.
+// unless c >= k and the k-th best earlier block scores >= own.
 #include <climits>
 #include <cmath>
 
@@ -48,6 +55,7 @@ __device__ __forceinline__ void insert(float (&ts)[KM], int (&ti)[KM], float s, 
 template <typename T, int D, int KM>
 __global__ void __launch_bounds__(kThreads) gate_kernel(Dims dm, const T* __restrict__ q,
                                                         const float* __restrict__ kbar,
+                                                        const float* __restrict__ own,
                                                         const int32_t* __restrict__ cu,
                                                         int32_t* __restrict__ idx, int* status) {
   extern __shared__ __align__(16) float gsm[];
@@ -147,12 +155,13 @@ __global__ void __launch_bounds__(kThreads) gate_kernel(Dims dm, const T* __rest
   }
 
   // Merge the four lists of each query: round r takes the best head.
-  const int hsel = valid ? min(dm.topk - 1, c) : 0;
+  const int need = hist_slots(dm);
+  float kth = -INFINITY;  // score of the k-th best earlier block (prefix variant)
   int sel[KM];
 #pragma unroll
   for (int r = 0; r < KM; ++r) {
     sel[r] = INT_MAX;
-    if (r < dm.topk - 1) {
+    if (r < need) {
       float bs = ts[0];
       int bi = ti[0], owner = part;
 #pragma unroll
@@ -175,9 +184,21 @@ __global__ void __launch_bounds__(kThreads) gate_kernel(Dims dm, const T* __rest
         ts[KM - 1] = -INFINITY;
         ti[KM - 1] = INT_MAX;
       }
-      if (r < hsel) sel[r] = bi;
+      if (r < c) sel[r] = bi;
+      if (r == dm.topk - 1) kth = bs;
     }
   }
+  // the own block: forced, or in unless k earlier blocks score at least as high
+  bool own_in = true;
+  if (dm.prefix && valid) {
+    float so = 0.f;
+    for (int hh = 0; hh < nh; ++hh) so += own[(start + p) * dm.Hq + h0 + hh];
+    own_in = !(c >= dm.topk && kth >= so);
+  }
+  const int hsel = valid ? (own_in ? min(dm.topk - 1, c) : dm.topk) : 0;
+#pragma unroll
+  for (int r = 0; r < KM; ++r)
+    if (r >= hsel) sel[r] = INT_MAX;
   if (part != 0 || !valid) return;
   // ascending order of the chosen earlier blocks
 #pragma unroll
@@ -195,47 +216,48 @@ __global__ void __launch_bounds__(kThreads) gate_kernel(Dims dm, const T* __rest
     int32_t* row = idx + ((start + p) * dm.Hq + h0 + hh) * (int64_t)dm.topk;
 #pragma unroll
     for (int r = 0; r <= KM; ++r) {
-      if (r < dm.topk) row[r] = r < hsel ? sel[r < KM ? r : KM - 1] : (r == hsel ? c : -1);
+      if (r < dm.topk)
+        row[r] = r < hsel ? sel[r < KM ? r : KM - 1] : (r == hsel && own_in ? c : -1);
     }
   }
 }
 
 template <typename T, int D, int KM>
-cudaError_t run(const Dims& dm, const void* q, const float* kbar, const int32_t* cu, int32_t* idx,
-                int* status, cudaStream_t st) {
+cudaError_t run(const Dims& dm, const void* q, const float* kbar, const float* own,
+                const int32_t* cu, int32_t* idx, int* status, cudaStream_t st) {
   dim3 grid((dm.max_seqlen + kQ - 1) / kQ, dm.batch, dm.shared ? dm.Hkv : dm.Hq);
   const size_t smem = sizeof(float) * ((kQ + kCh) * (D + 4) + kQ * (kCh + 1));
   cudaError_t e = cudaFuncSetAttribute(gate_kernel<T, D, KM>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  gate_kernel<T, D, KM><<<grid, kThreads, smem, st>>>(dm, static_cast<const T*>(q), kbar, cu,
-                                                      idx, status);
+  gate_kernel<T, D, KM><<<grid, kThreads, smem, st>>>(dm, static_cast<const T*>(q), kbar, own,
+                                                      cu, idx, status);
   return cudaGetLastError();
 }
 
 template <typename T, int D>
-cudaError_t by_k(const Dims& dm, const void* q, const float* kbar, const int32_t* cu, int32_t* idx,
-                 int* status, cudaStream_t st) {
-  const int need = dm.topk - 1;
-  if (need <= 1) return run<T, D, 1>(dm, q, kbar, cu, idx, status, st);
-  if (need <= 2) return run<T, D, 2>(dm, q, kbar, cu, idx, status, st);
-  if (need <= 4) return run<T, D, 4>(dm, q, kbar, cu, idx, status, st);
-  if (need <= 8) return run<T, D, 8>(dm, q, kbar, cu, idx, status, st);
-  if (need <= 16) return run<T, D, 16>(dm, q, kbar, cu, idx, status, st);
-  return run<T, D, 32>(dm, q, kbar, cu, idx, status, st);
+cudaError_t by_k(const Dims& dm, const void* q, const float* kbar, const float* own,
+                 const int32_t* cu, int32_t* idx, int* status, cudaStream_t st) {
+  const int need = hist_slots(dm);
+  if (need <= 1) return run<T, D, 1>(dm, q, kbar, own, cu, idx, status, st);
+  if (need <= 2) return run<T, D, 2>(dm, q, kbar, own, cu, idx, status, st);
+  if (need <= 4) return run<T, D, 4>(dm, q, kbar, own, cu, idx, status, st);
+  if (need <= 8) return run<T, D, 8>(dm, q, kbar, own, cu, idx, status, st);
+  if (need <= 16) return run<T, D, 16>(dm, q, kbar, own, cu, idx, status, st);
+  return run<T, D, 32>(dm, q, kbar, own, cu, idx, status, st);
 }
 
 }  // namespace
 
-cudaError_t launch_gate(const Dims& dm, const void* q, const float* kbar, const int32_t* cu,
-                        int32_t* idx, int* status, cudaStream_t st) {
+cudaError_t launch_gate(const Dims& dm, const void* q, const float* kbar, const float* own,
+                        const int32_t* cu, int32_t* idx, int* status, cudaStream_t st) {
   if (dm.batch == 0 || dm.max_seqlen == 0) return cudaSuccess;
-  if (gate_tc_supported(dm)) return launch_gate_tc(dm, q, kbar, cu, idx, status, st);
+  if (gate_tc_supported(dm)) return launch_gate_tc(dm, q, kbar, own, cu, idx, status, st);
   if (dm.dtype == kBF16)
-    return dm.d == 128 ? by_k<__nv_bfloat16, 128>(dm, q, kbar, cu, idx, status, st)
-                       : by_k<__nv_bfloat16, 64>(dm, q, kbar, cu, idx, status, st);
-  return dm.d == 128 ? by_k<float, 128>(dm, q, kbar, cu, idx, status, st)
-                     : by_k<float, 64>(dm, q, kbar, cu, idx, status, st);
+    return dm.d == 128 ? by_k<__nv_bfloat16, 128>(dm, q, kbar, own, cu, idx, status, st)
+                       : by_k<__nv_bfloat16, 64>(dm, q, kbar, own, cu, idx, status, st);
+  return dm.d == 128 ? by_k<float, 128>(dm, q, kbar, own, cu, idx, status, st)
+                     : by_k<float, 64>(dm, q, kbar, own, cu, idx, status, st);
 }
 
 }  // namespace moba

@@ -57,6 +57,10 @@ moba_status dims_of(const moba_params* p, moba::Dims& dm) {
       p->num_kv_heads <= 0 || p->num_q_heads % p->num_kv_heads != 0 || p->block_size <= 0 ||
       p->topk <= 0)
     return MOBA_ERR_INVALID_ARG;
+  if (p->routing != 0 && p->routing != 1) return MOBA_ERR_INVALID_ARG;
+  if (p->own_block != 0 && p->own_block != 1) return MOBA_ERR_INVALID_ARG;
+  // the prefix-mean gate keeps T * Hq own-block scores: no room in the fixed array
+  if (p->own_block) return MOBA_ERR_UNSUPPORTED;
   if (p->dtype != MOBA_BF16 && p->dtype != MOBA_F32) return MOBA_ERR_UNSUPPORTED;
   if (p->head_dim != 64 && p->head_dim != 128) return MOBA_ERR_UNSUPPORTED;
   if (p->topk > 32) return MOBA_ERR_UNSUPPORTED;
@@ -72,6 +76,8 @@ moba_status dims_of(const moba_params* p, moba::Dims& dm) {
   dm.topk = p->topk;
   dm.nb = (int)(((int64_t)p->max_seqlen + p->block_size - 1) / p->block_size);
   dm.dtype = p->dtype == MOBA_BF16 ? moba::kBF16 : moba::kF32;
+  dm.shared = p->routing;
+  dm.prefix = 0;
   return MOBA_OK;
 }
 
@@ -97,7 +103,7 @@ extern "C" moba_status moba_gate_topk_noalloc(const moba_params* p, const void* 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (moba::launch_meanpool(dm, k, cu_seqlens, kbar, nullptr, st) != cudaSuccess)
     return MOBA_ERR_CUDA;
-  if (moba::launch_gate(dm, q, kbar, cu_seqlens, idx, nullptr, st) != cudaSuccess)
+  if (moba::launch_gate(dm, q, kbar, nullptr, cu_seqlens, idx, nullptr, st) != cudaSuccess)
     return MOBA_ERR_CUDA;
   return MOBA_OK;
 }

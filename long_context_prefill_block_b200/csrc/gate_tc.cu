@@ -36,6 +36,7 @@ constexpr int kCuSmem = 257;                 // sequence offsets kept in shared 
 struct GateArgs {
   Dims dm;
   const float* kbar;
+  const float* own;  // own-block scores [T][Hq] of the prefix-mean gate, else unused
   const int32_t* cu;
   int32_t* idx;
   int* status;
@@ -358,7 +359,18 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmq, const GateArgs a) {
       }
     }
     if (part == 0 && valid) {
-      const int hsel = min(dm.topk - 1, c);
+      // the own block: forced, or (prefix mean) in unless k earlier blocks
+      // score at least as high; it loses ties, being the highest index
+      bool own_in = true;
+      if (dm.prefix && c >= dm.topk) {
+        float kth = -INFINITY, so = 0.f;
+#pragma unroll
+        for (int j = 0; j < KM; ++j)
+          if (j == dm.topk - 1) kth = ts[j];
+        for (int hh = 0; hh < nh; ++hh) so += a.own[(x.start + p) * dm.Hq + x.h + hh];
+        own_in = !(kth >= so);
+      }
+      const int hsel = own_in ? min(dm.topk - 1, c) : dm.topk;
       int sel[KM];
 #pragma unroll
       for (int r = 0; r < KM; ++r) sel[r] = r < hsel ? ti[r] : INT_MAX;
@@ -375,7 +387,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmq, const GateArgs a) {
       for (int hh = 0; hh < nh; ++hh) {
         int32_t* row = a.idx + ((x.start + p) * dm.Hq + x.h + hh) * (int64_t)dm.topk;
         for (int r = 0; r < dm.topk; ++r)
-          row[r] = r < hsel ? sel[r < KM ? r : KM - 1] : (r == hsel ? c : -1);
+          row[r] = r < hsel ? sel[r < KM ? r : KM - 1] : (r == hsel && own_in ? c : -1);
       }
     }
     // TMEM and this Q buffer are free again
@@ -449,12 +461,13 @@ bool gate_tc_supported(const Dims& dm) {
   return dm.dtype == kBF16 && dm.d == 128 && dm.nb <= kMaxBlocks && dm.topk <= 33;
 }
 
-cudaError_t launch_gate_tc(const Dims& dm, const void* q, const float* kbar, const int32_t* cu,
-                           int32_t* idx, int* status, cudaStream_t st) {
+cudaError_t launch_gate_tc(const Dims& dm, const void* q, const float* kbar, const float* own,
+                           const int32_t* cu, int32_t* idx, int* status, cudaStream_t st) {
   if (dm.batch == 0 || dm.max_seqlen == 0) return cudaSuccess;
   GateArgs a{};
   a.dm = dm;
   a.kbar = kbar;
+  a.own = own;
   a.cu = cu;
   a.idx = idx;
   a.status = status;
@@ -464,7 +477,7 @@ cudaError_t launch_gate_tc(const Dims& dm, const void* q, const float* kbar, con
   a.groups = dm.batch * dm.Hkv;
   a.ipg = (int)ipg;
   a.nbp = ((dm.nb + 15) / 16) * 16;
-  const int need = dm.topk - 1;
+  const int need = hist_slots(dm);
   const int km = need <= 1 ? 1 : need <= 2 ? 2 : need <= 4 ? 4 : need <= 8 ? 8 : need <= 16 ? 16 : 32;
   const size_t fixed = 1024 + (size_t)3 * 2 * a.nbp * 128;
   constexpr size_t kSmemMax = kMaxSmem;

@@ -13,8 +13,9 @@
 // so the order changes no output bit.
 //
 // The count pass also checks each index row's canonical form (strictly
-// ascending earlier blocks, then the own block c, then -1 padding) and
-// records kStBadIndices for a row that breaks it; such entries are skipped.
+// ascending earlier blocks, then the own block c, then -1 padding; with the
+// prefix-mean gate c may be absent) and records kStBadIndices for a row that
+// breaks it; such entries are skipped.
 #include "common.cuh"
 
 namespace moba {
@@ -24,17 +25,21 @@ constexpr int kThreads = 128;
 constexpr int kScanThreads = 1024;
 
 // Walks one index row; calls f(slot, block) for every history entry and
-// returns false if the row is not canonical.
+// returns false if the row is not canonical (own_required: block c must be
+// named).
 template <typename F>
-__device__ __forceinline__ bool walk_row(const int32_t* row, int topk, int c, F f) {
+__device__ __forceinline__ bool walk_row(const int32_t* row, int topk, int c, bool own_required,
+                                         F f) {
   int prev = -1;
-  bool seen_c = false, ok = true;
+  bool seen_c = false, seen_pad = false, ok = true;
   for (int r = 0; r < topk; ++r) {
     const int e = row[r];
-    if (seen_c) {
+    if (seen_c || seen_pad) {
       ok &= (e == -1);
     } else if (e == c) {
       seen_c = true;
+    } else if (e == -1) {
+      seen_pad = true;
     } else if (e >= 0 && e < c && e > prev) {
       prev = e;
       f(r, e);
@@ -42,7 +47,8 @@ __device__ __forceinline__ bool walk_row(const int32_t* row, int topk, int c, F 
       ok = false;
     }
   }
-  return ok && seen_c;
+  // a row without its own block must name at least one earlier block
+  return ok && (seen_c || (!own_required && prev >= 0));
 }
 
 template <bool SCATTER>
@@ -66,7 +72,7 @@ __global__ void __launch_bounds__(kThreads) regroup_pass(Dims dm, Chunk ch,
   const int32_t* row = idx + (t * dm.Hq + h) * (int64_t)dm.topk;
   const int list0 = (b * ch.ng + gl) * dm.nb;
   const int64_t prow0 = (t * ch.nq + hl) * (int64_t)dm.topk;
-  const bool ok = walk_row(row, dm.topk, c, [&](int slot, int e) {
+  const bool ok = walk_row(row, dm.topk, c, !dm.prefix, [&](int slot, int e) {
     if (SCATTER) {
       const int list = list0 + e;
       const int pos = atomicAdd(&cursor[list], 1);
@@ -116,7 +122,7 @@ __global__ void __launch_bounds__(kRows) regroup_pass_smem(Dims dm, Chunk ch,
   const int list0 = (b * ch.ng + gl) * dm.nb;
   const int64_t prow0 = (t * ch.nq + hl) * (int64_t)dm.topk;
   bool ok = true;
-  if (valid) ok = walk_row(row, dm.topk, c, [&](int, int e) { atomicAdd(&hist[e], 1); });
+  if (valid) ok = walk_row(row, dm.topk, c, !dm.prefix, [&](int, int e) { atomicAdd(&hist[e], 1); });
   if (!SCATTER && !ok) set_status(status, kStBadIndices);
   __syncthreads();
   for (int e = threadIdx.x; e < cmax; e += kRows) {
@@ -131,7 +137,7 @@ __global__ void __launch_bounds__(kRows) regroup_pass_smem(Dims dm, Chunk ch,
   if (!SCATTER) return;
   __syncthreads();
   if (valid)
-    walk_row(row, dm.topk, c, [&](int slot, int e) {
+    walk_row(row, dm.topk, c, !dm.prefix, [&](int slot, int e) {
       const int pos = base[e] + atomicAdd(&hist[e], 1);
       pairs[list_off[list0 + e] + pos] = (int32_t)(prow0 + slot);
     });

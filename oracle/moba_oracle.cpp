@@ -34,7 +34,7 @@
 //                             history branch and merges them with [PT §2]
 //                             eq. (7)-(8).
 //
-// Routing variant ([PT §5.4], the paragraph on multi-head settings: a group
+// Routing variant ([PT §5.5], the paragraph on multi-head settings: a group
 // of heads may share its candidate blocks, the routing score then has to
 // aggregate the heads' needs): with shared routing every query head of a kv
 // head's group gets the same blocks, chosen by the group's MEAN score

@@ -44,23 +44,24 @@ def index_mismatches(gpu_idx, ref_idx, gap):
 
 
 def check_forward(q, k, v, cu, B, topk, out_gpu, lse_gpu=None, idx_gpu=None, indices=None,
-                  shared_routing=False):
+                  shared_routing=False, prefix_mean=False):
     """Full oracle comparison of a forward result (small shapes)."""
     dtype = q.dtype
     ref, ref_lse, ref_idx, _ = oracle.forward(q.cpu(), k.cpu(), v.cpu(), cu.cpu(), B, topk,
                                               indices=None if indices is None else indices.cpu(),
-                                              shared_routing=shared_routing)
+                                              shared_routing=shared_routing,
+                                              prefix_mean=prefix_mean)
     out = out_gpu.float().cpu().numpy()
     T, Hq = q.shape[:2]
     if idx_gpu is not None and indices is None:
         _, gap = oracle.gate_topk(q.cpu(), k.cpu(), cu.cpu(), B, topk,
-                                  shared_routing=shared_routing)
+                                  shared_routing=shared_routing, prefix_mean=prefix_mean)
         bad = index_mismatches(idx_gpu.cpu().numpy(), ref_idx, gap)
         if len(bad):
             # near-tie rows: the oracle with the GPU's own choice
             gi = idx_gpu.cpu().numpy().reshape(T * Hq, topk)[bad]
             o2, l2, _, _ = oracle.forward_rows(q.cpu(), k.cpu(), v.cpu(), cu.cpu(), B, topk, bad,
-                                               indices=gi)
+                                               indices=gi, prefix_mean=prefix_mean)
             ref = ref.reshape(T * Hq, -1).copy()
             ref[bad] = o2
             ref = ref.reshape(out.shape)
@@ -74,19 +75,21 @@ def check_forward(q, k, v, cu, B, topk, out_gpu, lse_gpu=None, idx_gpu=None, ind
     return ref
 
 
-def check_rows(q, k, v, cu, B, topk, rows, out_gpu, idx_gpu=None, lse_gpu=None):
+def check_rows(q, k, v, cu, B, topk, rows, out_gpu, idx_gpu=None, lse_gpu=None,
+               prefix_mean=False):
     """Sampled oracle comparison on flattened rows (row = t * Hq + h)."""
     dtype = q.dtype
     T, Hq, d = q.shape
     qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
     rows = np.asarray(rows, dtype=np.int64)
-    ref, ref_lse, ref_idx, gap = oracle.forward_rows(qc, kc, vc, cu.cpu(), B, topk, rows)
+    ref, ref_lse, ref_idx, gap = oracle.forward_rows(qc, kc, vc, cu.cpu(), B, topk, rows,
+                                                     prefix_mean=prefix_mean)
     if idx_gpu is not None:
         gi = idx_gpu.reshape(T * Hq, topk)[torch.as_tensor(rows, device=idx_gpu.device)].cpu().numpy()
         bad = index_mismatches(gi, ref_idx, gap)
         if len(bad):
             o2, l2, _, _ = oracle.forward_rows(qc, kc, vc, cu.cpu(), B, topk, rows[bad],
-                                               indices=gi[bad])
+                                               indices=gi[bad], prefix_mean=prefix_mean)
             ref[bad] = o2
             ref_lse[bad] = l2
     sel = torch.as_tensor(rows, device=out_gpu.device)

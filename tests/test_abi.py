@@ -43,6 +43,19 @@ def params(**kw):
 
 def test_workspace_sizes():
     assert moba.moba_workspace_size(params()) > 0
+
+
+def test_prefix_mean_gate_workspace():
+    # the prefix-mean gate keeps one fp32 own-block score per (token, q head)
+    # and up to k history entries per row instead of k - 1
+    base, pref = params(), params(own_block=1)
+    extra = moba.moba_workspace_size(pref) - moba.moba_workspace_size(base)
+    assert extra >= 32768 * 32 * 4
+    # the allocation-free gate has no room for those scores: refused before any launch
+    fn = moba.lib().moba_gate_topk_noalloc
+    fn.argtypes = [ctypes.POINTER(moba.MobaParams)] + [ctypes.c_void_p] * 5
+    fn.restype = ctypes.c_int
+    assert fn(ctypes.byref(pref), None, None, None, None, None) == moba.MOBA_ERR_UNSUPPORTED
     # million-token GQA shape: partial results are kept one kv-head group at a time
     big = params(total_tokens=1 << 20, max_seqlen=1 << 20, num_kv_heads=8, block_size=4096, topk=12)
     assert 0 < moba.moba_workspace_size(big) < 48 * (1 << 30)
@@ -51,7 +64,7 @@ def test_workspace_sizes():
 
 @pytest.mark.parametrize("bad", [
     dict(num_q_heads=3, num_kv_heads=2), dict(block_size=0), dict(topk=0), dict(batch=-1),
-    dict(routing=2), dict(routing=-1),
+    dict(routing=2), dict(routing=-1), dict(own_block=2), dict(own_block=-1),
     dict(num_kv_heads=0)])
 def test_invalid_params_rejected(bad):
     p = params(**bad)

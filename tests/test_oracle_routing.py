@@ -1,5 +1,5 @@
 """Pins of the oracle's shared-routing variant (PaperTrace "2.1.3 MoBA",
-section 5.4, multi-head settings: the query heads of a group share their
+section 5.5, multi-head settings: the query heads of a group share their
 candidate blocks, chosen on the group's mean score). Each pin reduces the
 variant to the per-head gate, which tests/test_oracle_pins.py pins to the
 pages' worked example, brute force and closed forms."""
