@@ -2,7 +2,8 @@
 """Benchmark of the B200 MoBA prefill forward pass (one layer-forward = one step).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
-                    [--variant forced|shared|prefix] [--pass forward|backward]
+                    [--variant forced|shared|prefix] [--pass forward|backward|decode]
+                    [--queries N]
 
 A step runs the whole path -- block mean-pool, gate/top-k, regrouping,
 history and own-block attention, merge -- on seeded synthetic inputs of the
@@ -25,7 +26,10 @@ own block scored by the mean of its keys up to the query). Useful FLOPs of
 the prefix variant are counted from the gate's own index rows. --pass
 backward times moba_backward (dq, dk, dv through the chosen blocks, on the
 forward's indices): useful FLOPs 2.5x the forward's (five contractions per
-query-key pair against two).
+query-key pair against two). --pass decode times one decode step
+(moba_decode: every request's last --queries positions against its cache,
+the workload's K/V) in microseconds, with the bytes it must read (the chosen
+keys' K and V, the scored block means, q and out) against the HBM peak.
 """
 from __future__ import annotations
 
@@ -343,6 +347,134 @@ def bench_backward(args, w, moba, q, k, v, cu, dev, world, rank, config, shared,
         torch.distributed.destroy_process_group()
 
 
+def bench_decode(args, w, moba, q_all, k, v, cu, dev, world, rank, config, shared):
+    """--pass decode: one decode step = every request's last --queries positions against its
+    cache (the workload's K/V), through moba_decode; the block means are built once, as a
+    serving loop keeps them up to date incrementally."""
+    nq_r = args.queries
+    lens = np.diff(cu.numpy())
+    if (lens < nq_r).any():
+        raise ValueError("--queries exceeds a sequence length")
+    Hq, d = q_all.shape[1], q_all.shape[2]
+    tok = torch.cat([torch.arange(int(cu[r + 1]) - nq_r, int(cu[r + 1])) for r in range(w.batch)])
+    q = q_all[tok.to(dev)].contiguous()
+    del q_all
+    cu_d = cu.to(dev)
+    cu_q = torch.arange(0, (w.batch + 1) * nq_r, nq_r, dtype=torch.int32)
+    kbar = moba.moba_meanpool(k, cu_d, w.block_size, max_seqlen=w.max_seqlen)
+    p = moba.decode_params(q, k, cu, w.block_size, w.topk, w.max_seqlen, shared)
+    L = moba.lib()
+    L.moba_decode_workspace_size.argtypes = [ctypes.POINTER(moba.MobaParams), ctypes.c_int]
+    L.moba_decode_workspace_size.restype = ctypes.c_size_t
+    n = q.shape[0]
+    ws = torch.empty(max(int(L.moba_decode_workspace_size(ctypes.byref(p), n)), 256),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    idx = torch.empty((n, Hq, w.topk), dtype=torch.int32, device=dev)
+    cu_qd = cu_q.to(dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    fn = L.moba_decode
+    V = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(moba.MobaParams), V, V, V, V, V, ctypes.c_int, V, V, V, V, V,
+                   ctypes.c_size_t, V]
+    fn.restype = ctypes.c_int
+    P = ctypes.byref(p)
+    ptr = lambda x: ctypes.c_void_p(x.data_ptr())
+
+    def step(qq=q, oo=out):
+        rc = fn(P, ptr(qq), ptr(k), ptr(v), ptr(cu_d), ptr(cu_qd), n, ptr(kbar), ptr(oo), None,
+                ptr(idx), ptr(ws), ws.numel(), sp)
+        if rc:
+            raise RuntimeError(f"moba_decode failed: {rc}")
+
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    if clocks:
+        clocks.wait_first_sample()
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    if moba.moba_device_status(dev) != 0:
+        raise RuntimeError("device status error after warm-up")
+    # bytes the step must read: the chosen keys' K and V rows of every (query, q head), the
+    # block means it scores and the query rows (output written once)
+    pos = (torch.as_tensor(lens, device=dev).repeat_interleave(nq_r) - nq_r
+           + torch.arange(nq_r, device=dev).repeat(w.batch))  # [n] positions
+    c = (pos // w.block_size)[:, None, None]
+    nkeys = (((idx >= 0) & (idx < c)).sum() * w.block_size
+             + (((pos - (pos // w.block_size) * w.block_size + 1)[:, None]) * (idx == c).any(2)).sum())
+    esz = k.element_size()
+    kv_bytes = int(nkeys.item()) * 2 * d * esz
+    gate_bytes = int((pos // w.block_size).sum().item()) * (Hq if not shared else w.num_kv_heads) * d * 4
+    io_bytes = 2 * q.numel() * esz
+    alg_bytes = kv_bytes + gate_bytes + io_bytes
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t_lo = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_hi = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    if clocks:
+        clocks.stop()
+    clock_info = clocks.summarise(t_lo, t_hi) if clocks else None
+    ms = reduce_max(e0.elapsed_time(e1) / args.steps, world, dev)
+    # end to end: the step's query rows in from pinned memory, the outputs back
+    hq = q.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq = torch.empty_like(q)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        step(dq, out)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    erep = max(3, min(args.steps, 20))
+    e0.record(stream)
+    for _ in range(erep):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / erep, world, dev)
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    achieved = alg_bytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": "moba_decode_step_us", "value": ms * 1e3, "unit": "us",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": dict(config, **{"pass": "decode", "queries_per_request": nq_r}),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "kernel": "moba_decode, all launches (gate, split-K attention with the merge)",
+                     "algorithmic_bytes": alg_bytes, "peak_source": f"{peak_src} HBM copy"},
+        "cpu_baseline": None,
+        "e2e": {"value": e2e_ms * 1e3, "unit": "us", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": hq.numel() * hq.element_size(),
+                "d2h_bytes_per_step": hout.numel() * hout.element_size()},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clock_info,
+        "queries_per_step": n,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -353,7 +485,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", default="forced", choices=["forced", "shared", "prefix"])
-    ap.add_argument("--pass", dest="pass_", default="forward", choices=["forward", "backward"])
+    ap.add_argument("--pass", dest="pass_", default="forward",
+                    choices=["forward", "backward", "decode"])
+    ap.add_argument("--queries", type=int, default=1, help="decode: queries per request")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -407,6 +541,10 @@ def main():
     shared, prefix = args.variant == "shared", args.variant == "prefix"
     if args.pass_ == "backward":
         return bench_backward(args, w, moba, q, k, v, cu, dev, world, rank, config, shared, prefix)
+    if args.pass_ == "decode":
+        if prefix:
+            raise ValueError("the decode step takes the forced own block only")
+        return bench_decode(args, w, moba, q, k, v, cu, dev, world, rank, config, shared)
     p = moba.make_params(q, k, cu, w.block_size, w.topk, w.max_seqlen, shared, prefix)
     ws = moba.workspace(p, dev)
     if prefix:

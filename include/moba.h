@@ -201,6 +201,48 @@ MOBA_API moba_status moba_backward(const moba_params* p, const void* q, const vo
                                    float* dq, float* dk, float* dv, void* ws, size_t ws_bytes,
                                    void* stream);
 
+/* Decode step (PaperTrace "2.1.3 MoBA", section 5.1 on long outputs:
+ * incremental block means and logical block numbers; section 5.4: a decode
+ * step asks few queries and is bound by the KV reads and the launches).
+ * The KV cache holds, per request r, keys and values packed as in a prefill
+ * batch: tokens cu_seqlens[r] .. cu_seqlens[r+1]-1, cache length L_r (the new
+ * tokens' keys and values already appended). Request r asks
+ * n_r = cu_q[r+1] - cu_q[r] queries (1 for plain decoding, more for a
+ * speculative draft): the queries of its last positions L_r - n_r .. L_r - 1,
+ * in order. Every query gets exactly the prefill forward's result for its
+ * position (gate over the complete earlier blocks, own block forced, top-k,
+ * one softmax over the chosen keys, causal in the own block). Block ids are
+ * logical: block i of a request is its positions iB .. iB+B-1.
+ *   p: batch = requests, total_tokens = cache tokens, max_seqlen = the
+ *      longest cache; routing as in the prefill; own_block must be 0
+ *      (MOBA_ERR_UNSUPPORTED otherwise).
+ *   q: [n_queries][Hq][d] (p->dtype); k_cache, v_cache: [total_tokens][Hkv][d];
+ *   cu_seqlens, cu_q: device int32 [batch + 1]; cu_q[batch] = n_queries and
+ *      0 <= n_r <= L_r (else MOBA_ERR_INVALID_ARG in the status word).
+ *   kbar: fp32 [batch][moba_num_blocks(p)][Hkv][d], the cache's block means
+ *      (moba_meanpool once, then moba_meanpool_update after each append);
+ *      only complete blocks before each query's own block are read.
+ *   out: [n_queries][Hq][d] (p->dtype); lse: fp32 [n_queries][Hq] or NULL;
+ *   idx: int32 [n_queries][Hq][k] receives the chosen blocks (canonical
+ *      form), or NULL.
+ *   ws: moba_decode_workspace_size(p, n_queries) bytes, 16-byte aligned. */
+MOBA_API size_t moba_decode_workspace_size(const moba_params* p, int n_queries);
+MOBA_API moba_status moba_decode(const moba_params* p, const void* q, const void* k_cache,
+                                 const void* v_cache, const int32_t* cu_seqlens,
+                                 const int32_t* cu_q, int n_queries, const float* kbar, void* out,
+                                 float* lse, int32_t* idx, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/* Incremental block means (section 5.1): after n_r = cu_new[r+1] - cu_new[r]
+ * tokens were appended to request r's cache (cu_seqlens describing the cache
+ * after the append), recomputes, exactly as moba_meanpool would, the entries
+ * of kbar for the blocks that hold positions L_r - n_r .. L_r - 1, and leaves
+ * every other entry untouched. max_new >= max_r n_r bounds the launch.
+ * cu_new: device int32 [batch + 1]. */
+MOBA_API moba_status moba_meanpool_update(const moba_params* p, const void* k_cache,
+                                          const int32_t* cu_seqlens, const int32_t* cu_new,
+                                          int max_new, float* kbar, void* stream);
+
 /* Dense causal softmax attention, eq. (1) with a causal mask (every key
  * j <= p of the query's own sequence), for comparison and for the full
  * budget limit (section 4). block_size and topk in p must be valid but do

@@ -141,6 +141,72 @@ def moba_meanpool(k: torch.Tensor, cu_seqlens: torch.Tensor, block_size: int,
     return kbar
 
 
+def moba_meanpool_update(k_cache: torch.Tensor, cu_seqlens: torch.Tensor, cu_new: torch.Tensor,
+                         kbar: torch.Tensor, block_size: int, max_new: int,
+                         max_seqlen: Optional[int] = None) -> torch.Tensor:
+    """Recompute, in place, the block means kbar [batch, num_blocks, Hkv, d] of the blocks that
+    hold each request's last cu_new[r+1] - cu_new[r] cache positions (just appended)."""
+    _check_inputs(k_cache, kbar)
+    p = make_params(k_cache, k_cache, cu_seqlens, block_size, 1, max_seqlen)
+    p.num_q_heads = p.num_kv_heads
+    cu = _dev_i32(cu_seqlens, k_cache.device)
+    cn = _dev_i32(cu_new, k_cache.device)
+    fn = lib().moba_meanpool_update
+    fn.argtypes = [ctypes.POINTER(MobaParams)] + [ctypes.c_void_p] * 3 + [ctypes.c_int,
+                                                                        ctypes.c_void_p,
+                                                                        ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check("moba_meanpool_update", fn(ctypes.byref(p), _ptr(k_cache), _ptr(cu), _ptr(cn),
+                                      int(max_new), _ptr(kbar), _stream(k_cache.device)))
+    return kbar
+
+
+def decode_params(q, k_cache, cu_seqlens, block_size: int, topk: int, max_seqlen=None,
+                  shared_routing: bool = False) -> MobaParams:
+    """Parameters of a decode step: the cache's shape with q's heads."""
+    p = make_params(k_cache, k_cache, cu_seqlens, block_size, topk, max_seqlen, shared_routing)
+    p.num_q_heads = q.shape[1]
+    return p
+
+
+def moba_decode(q, k_cache, v_cache, cu_seqlens, cu_q, kbar, block_size: int, topk: int,
+                max_seqlen=None, shared_routing: bool = False, return_lse: bool = False,
+                return_idx: bool = False, ws: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None):
+    """Decode step: request r's queries (rows cu_q[r] .. cu_q[r+1]-1 of q [n, Hq, d]) sit at the
+    last positions of its cache (tokens cu_seqlens[r] .. cu_seqlens[r+1]-1 of k_cache, v_cache);
+    kbar: the cache's block means. Returns out [n, Hq, d] (and lse [n, Hq], idx [n, Hq, topk])."""
+    _check_inputs(q, k_cache, v_cache, kbar)
+    L = lib()
+    p = decode_params(q, k_cache, cu_seqlens, block_size, topk, max_seqlen, shared_routing)
+    n = q.shape[0]
+    cu = _dev_i32(cu_seqlens, q.device)
+    cq = _dev_i32(cu_q, q.device)
+    L.moba_decode_workspace_size.argtypes = [ctypes.POINTER(MobaParams), ctypes.c_int]
+    L.moba_decode_workspace_size.restype = ctypes.c_size_t
+    if ws is None:
+        ws = torch.empty(max(int(L.moba_decode_workspace_size(ctypes.byref(p), n)), 256),
+                         dtype=torch.uint8, device=q.device)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device) if return_lse else None
+    idx = (torch.empty((n, q.shape[1], topk), dtype=torch.int32, device=q.device)
+           if return_idx else None)
+    fn = L.moba_decode
+    V = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(MobaParams), V, V, V, V, V, ctypes.c_int, V, V, V, V, V,
+                   ctypes.c_size_t, V]
+    fn.restype = ctypes.c_int
+    _check("moba_decode", fn(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cu),
+                             _ptr(cq), n, _ptr(kbar), _ptr(out), _ptr(lse), _ptr(idx), _ptr(ws),
+                             ws.numel(), _stream(q.device)))
+    res = (out,)
+    if return_lse:
+        res += (lse,)
+    if return_idx:
+        res += (idx,)
+    return res[0] if len(res) == 1 else res
+
+
 def moba_gate_topk(q, k, cu_seqlens, block_size: int, topk: int, max_seqlen=None,
                    ws: Optional[torch.Tensor] = None, shared_routing: bool = False,
                    prefix_mean: bool = False) -> torch.Tensor:

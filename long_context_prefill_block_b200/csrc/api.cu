@@ -320,9 +320,83 @@ moba_status backward_impl(const moba_params* p, const void* q, const void* k, co
   return MOBA_OK;
 }
 
+// Decode workspace: index rows, the split partials (o, then lse), the
+// per-row arrival counters.
+struct DecLayout {
+  size_t idx, part_o, part_lse, arrivals, total;
+};
+
+DecLayout plan_decode(const Dims& dm, int n_queries) {
+  DecLayout L{};
+  const size_t rows = decode_partial_rows(dm, n_queries);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L.idx = take(sizeof(int32_t) * (size_t)n_queries * dm.Hq * dm.topk);
+  L.part_o = take(sizeof(float) * rows * dm.d);
+  L.part_lse = take(sizeof(float) * rows);
+  L.arrivals = take(sizeof(int) * (size_t)n_queries * dm.Hq);
+  L.total = off;
+  return L;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t moba_decode_workspace_size(const moba_params* p, int n_queries) {
+  Dims dm;
+  if (validate(p, dm) != MOBA_OK || n_queries < 0) return 0;
+  return plan_decode(dm, n_queries).total;
+}
+
+moba_status moba_decode(const moba_params* p, const void* q, const void* k_cache,
+                        const void* v_cache, const int32_t* cu_seqlens, const int32_t* cu_q,
+                        int n_queries, const float* kbar, void* out, float* lse, int32_t* idx,
+                        void* ws, size_t ws_bytes, void* stream) {
+  Dims dm;
+  moba_status s = validate(p, dm);
+  if (s != MOBA_OK) return s;
+  if (n_queries < 0) return MOBA_ERR_INVALID_ARG;
+  if (dm.prefix) return MOBA_ERR_UNSUPPORTED;
+  if (dm.batch == 0 || n_queries == 0) return MOBA_OK;
+  if ((int64_t)n_queries * dm.Hq * dm.topk >= (int64_t(1) << 31)) return MOBA_ERR_UNSUPPORTED;
+  if (!q || !k_cache || !v_cache || !cu_seqlens || !cu_q || !kbar || !out)
+    return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(kbar) ||
+      !aligned16(out))
+    return MOBA_ERR_INVALID_ARG;
+  const DecLayout L = plan_decode(dm, n_queries);
+  if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOBA_ERR_WORKSPACE;
+  int* status = status_word();
+  if (!status) return MOBA_ERR_CUDA;
+  char* base = static_cast<char*>(ws);
+  int32_t* rows = idx ? idx : reinterpret_cast<int32_t*>(base + L.idx);
+  return cuda_status(launch_decode(dm, n_queries, q, k_cache, v_cache, cu_seqlens, cu_q, kbar, rows,
+                                   reinterpret_cast<float*>(base + L.part_o),
+                                   reinterpret_cast<float*>(base + L.part_lse),
+                                   reinterpret_cast<int*>(base + L.arrivals), out, lse, status,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+moba_status moba_meanpool_update(const moba_params* p, const void* k_cache,
+                                 const int32_t* cu_seqlens, const int32_t* cu_new, int max_new,
+                                 float* kbar, void* stream) {
+  Dims dm;
+  moba_status s = validate(p, dm);
+  if (s != MOBA_OK) return s;
+  if (max_new < 0) return MOBA_ERR_INVALID_ARG;
+  if (dm.batch == 0 || dm.nb == 0 || max_new == 0) return MOBA_OK;
+  if (!k_cache || !cu_seqlens || !cu_new || !kbar || !aligned16(k_cache) || !aligned16(kbar))
+    return MOBA_ERR_INVALID_ARG;
+  int* status = status_word();
+  if (!status) return MOBA_ERR_CUDA;
+  return cuda_status(launch_meanpool_update(dm, k_cache, cu_seqlens, cu_new, max_new, kbar, status,
+                                            static_cast<cudaStream_t>(stream)));
+}
 
 int moba_num_blocks(const moba_params* p) {
   Dims dm;

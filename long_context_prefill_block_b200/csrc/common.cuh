@@ -122,6 +122,19 @@ namespace moba {
 
 cudaError_t launch_meanpool(const Dims& dm, const void* k, const int32_t* cu, float* kbar,
                             int* status, cudaStream_t st);
+// Block means of only the blocks holding each sequence's last
+// cu_new[b+1] - cu_new[b] positions (max_new: the largest such count).
+cudaError_t launch_meanpool_update(const Dims& dm, const void* k, const int32_t* cu,
+                                   const int32_t* cu_new, int max_new, float* kbar, int* status,
+                                   cudaStream_t st);
+// Decode step (decode.cu): gate into idx, split-K attention into partials
+// [decode_partial_rows] x (d + 1) merged by the last split of each row into
+// out / lse; arrivals: n_queries * Hq ints of scratch (zeroed by the gate).
+size_t decode_partial_rows(const Dims& dm, int n_queries);
+cudaError_t launch_decode(const Dims& dm, int n_queries, const void* q, const void* k,
+                          const void* v, const int32_t* cu, const int32_t* cu_q, const float* kbar,
+                          int32_t* idx, float* part_o, float* part_lse, int* arrivals, void* out,
+                          float* lse, int* status, cudaStream_t st);
 // Tensor-core gate (bf16, d = 128, at most 256 blocks per sequence).
 bool gate_tc_supported(const Dims& dm);
 cudaError_t launch_gate_tc(const Dims& dm, const void* q, const float* kbar, const float* own,

@@ -7,6 +7,11 @@
 // threads, so every warp load is contiguous 128-256 B. Rows of one block are
 // spread over the CTA's row groups, summed in registers and reduced once in
 // shared memory: K is read exactly once (HBM-bound).
+//
+// Incremental form (section 5.1, long outputs need incremental means): with
+// cu_new, sequence b only recomputes the blocks that hold its last
+// n_b = cu_new[b+1] - cu_new[b] positions (the tokens just appended to its
+// cache); CTA x of the sequence takes the x-th of those blocks.
 #include "common.cuh"
 
 namespace moba {
@@ -17,6 +22,7 @@ constexpr int kThreads = 256;
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) meanpool_kernel(Dims dm, const T* __restrict__ k,
                                                             const int32_t* __restrict__ cu,
+                                                            const int32_t* __restrict__ cu_new,
                                                             float* __restrict__ kbar,
                                                             int* status) {
   constexpr int VEC = Vec16<T>::N;   // elements per 16-byte load
@@ -24,10 +30,22 @@ __global__ void __launch_bounds__(kThreads) meanpool_kernel(Dims dm, const T* __
   constexpr int RG = kThreads / TPR; // rows in flight
   __shared__ float red[RG][D + 1];
 
-  const int i = blockIdx.x, b = blockIdx.y, g = blockIdx.z;
+  const int b = blockIdx.y, g = blockIdx.z;
+  int i = blockIdx.x;
   int64_t start;
   int len;
   const bool ok = seq_bounds(dm, cu, b, start, len, status);
+  if (cu_new) {
+    if (!ok) return;
+    const int n = cu_new[b + 1] - cu_new[b];
+    if (n < 0 || n > len) {
+      set_status(status, kStInvalidArg);
+      return;
+    }
+    if (n == 0) return;
+    i += (len - n) / dm.B;
+    if (i * dm.B >= len) return;
+  }
   const int j0 = i * dm.B;
   const int j1 = ok ? min(len, j0 + dm.B) : j0;
   const int lane = threadIdx.x % TPR, rg = threadIdx.x / TPR;
@@ -54,23 +72,38 @@ __global__ void __launch_bounds__(kThreads) meanpool_kernel(Dims dm, const T* __
 }
 
 template <typename T, int D>
-cudaError_t run(const Dims& dm, const void* k, const int32_t* cu, float* kbar, int* status,
-                cudaStream_t st) {
-  dim3 grid(dm.nb, dm.batch, dm.Hkv);
-  meanpool_kernel<T, D><<<grid, kThreads, 0, st>>>(dm, static_cast<const T*>(k), cu, kbar, status);
+cudaError_t run(const Dims& dm, const void* k, const int32_t* cu, const int32_t* cu_new,
+                int nblk, float* kbar, int* status, cudaStream_t st) {
+  dim3 grid(nblk, dm.batch, dm.Hkv);
+  meanpool_kernel<T, D><<<grid, kThreads, 0, st>>>(dm, static_cast<const T*>(k), cu, cu_new, kbar,
+                                                   status);
   return cudaGetLastError();
+}
+
+cudaError_t launch(const Dims& dm, const void* k, const int32_t* cu, const int32_t* cu_new,
+                   int nblk, float* kbar, int* status, cudaStream_t st) {
+  if (dm.batch == 0 || nblk == 0) return cudaSuccess;
+  if (dm.dtype == kBF16)
+    return dm.d == 128 ? run<__nv_bfloat16, 128>(dm, k, cu, cu_new, nblk, kbar, status, st)
+                       : run<__nv_bfloat16, 64>(dm, k, cu, cu_new, nblk, kbar, status, st);
+  return dm.d == 128 ? run<float, 128>(dm, k, cu, cu_new, nblk, kbar, status, st)
+                     : run<float, 64>(dm, k, cu, cu_new, nblk, kbar, status, st);
 }
 
 }  // namespace
 
 cudaError_t launch_meanpool(const Dims& dm, const void* k, const int32_t* cu, float* kbar,
                             int* status, cudaStream_t st) {
-  if (dm.batch == 0 || dm.nb == 0) return cudaSuccess;
-  if (dm.dtype == kBF16)
-    return dm.d == 128 ? run<__nv_bfloat16, 128>(dm, k, cu, kbar, status, st)
-                       : run<__nv_bfloat16, 64>(dm, k, cu, kbar, status, st);
-  return dm.d == 128 ? run<float, 128>(dm, k, cu, kbar, status, st)
-                     : run<float, 64>(dm, k, cu, kbar, status, st);
+  return launch(dm, k, cu, nullptr, dm.nb, kbar, status, st);
+}
+
+cudaError_t launch_meanpool_update(const Dims& dm, const void* k, const int32_t* cu,
+                                   const int32_t* cu_new, int max_new, float* kbar, int* status,
+                                   cudaStream_t st) {
+  if (max_new <= 0) return cudaSuccess;
+  // n new positions touch at most ceil((n - 1) / B) + 1 blocks
+  const int64_t nblk = (int64_t)(max_new - 1) / dm.B + 2;
+  return launch(dm, k, cu, cu_new, (int)(nblk < dm.nb ? nblk : dm.nb), kbar, status, st);
 }
 
 }  // namespace moba

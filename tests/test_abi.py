@@ -106,3 +106,29 @@ def test_status_strings():
     lib = moba.lib()
     for code in (0, -1, -2, -3, -4, -5, -6):
         assert lib.moba_status_string(code)
+
+
+def test_decode_argument_checks():
+    # validated on the host before any launch: no GPU needed
+    L = moba.lib()
+    L.moba_decode_workspace_size.argtypes = [ctypes.POINTER(moba.MobaParams), ctypes.c_int]
+    L.moba_decode_workspace_size.restype = ctypes.c_size_t
+    assert L.moba_decode_workspace_size(ctypes.byref(params()), 4) > 0
+    assert L.moba_decode_workspace_size(ctypes.byref(params()), -1) == 0
+    fn = L.moba_decode
+    V = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(moba.MobaParams), V, V, V, V, V, ctypes.c_int, V, V, V, V, V,
+                   ctypes.c_size_t, V]
+    fn.restype = ctypes.c_int
+    args = [None] * 5
+    assert fn(ctypes.byref(params()), *args, -1, None, None, None, None, None, 0, None) \
+        == moba.MOBA_ERR_INVALID_ARG
+    assert fn(ctypes.byref(params(own_block=1)), *args, 1, None, None, None, None, None, 0, None) \
+        == moba.MOBA_ERR_UNSUPPORTED
+    assert fn(ctypes.byref(params()), *args, 0, None, None, None, None, None, 0, None) == moba.MOBA_OK
+    up = L.moba_meanpool_update
+    up.argtypes = [ctypes.POINTER(moba.MobaParams), V, V, V, ctypes.c_int, V, V]
+    up.restype = ctypes.c_int
+    assert up(ctypes.byref(params()), None, None, None, -1, None, None) == moba.MOBA_ERR_INVALID_ARG
+    assert up(ctypes.byref(params()), None, None, None, 0, None, None) == moba.MOBA_OK
+
