@@ -125,8 +125,9 @@ Layout plan(const Dims& dm, bool own_idx) {
   L.tile_off = take(sizeof(int32_t) * (n_lists + 1));
   L.pairs = take(sizeof(int32_t) * max_pairs);
   L.tiles = take(sizeof(int2) * L.max_tiles);
-  L.part_o = take(sizeof(float) * (size_t)dm.T * L.ng * grp * dm.topk * dm.d);
-  L.part_lse = take(sizeof(float) * (size_t)dm.T * L.ng * grp * dm.topk);
+  const size_t prows = part_rows(dm.T, (int64_t)L.ng * grp * dm.topk);
+  L.part_o = take(sizeof(float) * prows * dm.d);
+  L.part_lse = take(sizeof(float) * prows);
   L.total = off;
   return L;
 }

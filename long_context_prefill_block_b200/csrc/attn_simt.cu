@@ -193,13 +193,15 @@ attn_simt(Dims dm, Chunk ch, const T* __restrict__ q, const T* __restrict__ k,
       for (int u = 0; u < 4; ++u) dst[part * 4 + 16 * j + u] = from_f32<T>(o[j * 4 + u] * inv_l);
     if (lse_out && part == 0) lse_out[t * dm.Hq + h] = lse;
   } else {
-    float* dst = part_o + prow * D;
+    const PartRow pr = part_row(prow, (int64_t)ch.nq * dm.topk);
 #pragma unroll
-    for (int j = 0; j < NG; ++j)
-      *reinterpret_cast<float4*>(dst + part * 4 + 16 * j) =
+    for (int j = 0; j < NG; ++j) {
+      const int x0 = part * 4 + 16 * j;  // four columns inside one 8-column piece
+      *reinterpret_cast<float4*>(part_piece(part_o, pr, D, x0 / 8) + x0 % 8) =
           make_float4(o[j * 4] * inv_l, o[j * 4 + 1] * inv_l, o[j * 4 + 2] * inv_l,
                       o[j * 4 + 3] * inv_l);
-    if (part == 0) part_lse[prow] = lse;
+    }
+    if (part == 0) part_lse[part_lse_at(pr)] = lse;
   }
 }
 

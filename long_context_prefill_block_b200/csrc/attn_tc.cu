@@ -76,7 +76,6 @@ constexpr uint32_t kQOff = 0;          // Q[2], one per query half
 constexpr uint32_t kKOff = 2 * kTile;  // K[NS]
 constexpr uint32_t kVOff = kKOff + NS * kTile;
 constexpr uint32_t kStageRow = 80;     // bytes per staged row chunk: 64 + 16 pad
-constexpr uint32_t kStageRow128 = 144; // 128-byte row pieces, 16 rows at a time (fits 32 x 80)
 constexpr uint32_t kStageOff = kVOff + NS * kTile;  // epilogue staging, 32 rows per softmax warp
 constexpr uint32_t kStageBytes = 8 * 32 * kStageRow;
 constexpr uint32_t kSmemBytes = kStageOff + kStageBytes + 1024;  // + 1024-byte alignment slack
@@ -598,9 +597,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
         // (eq. 7-8 written with lse: w_j = exp(lse_j - m), o = sum_j w_j o_j /
         // sum_j w_j) and write the output; the own result never leaves the
         // SM. Slots 0..slot-1 of the row hold the history partials. Each
-        // thread merges its own row with 32 independent 16-byte loads per
-        // slot in flight. A row whose own block lost the prefix-mean gate
-        // gives its own result weight 0.
+        // thread merges its own row; the warp's 32 rows are 32 consecutive
+        // tokens of one head, so in the interleaved partial layout every
+        // 32-byte piece load of the warp is one contiguous 1 KB access. A
+        // row whose own block lost the prefix-mean gate gives its own result
+        // weight 0.
         const int slot = R.valid ? R.nhist : 0;
         const int64_t prow0 = R.valid ? R.prow : 0;
         const int64_t orow = R.valid ? R.t * dm.Hq + R.h : -1;
@@ -617,22 +618,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
         fence_before_sync();
         mbar_arrive(&sh.o_free[hh]);
         if (R.valid) {
+          const int64_t nr = (int64_t)a.ch.nq * dm.topk;
           float m = R.own ? lse : -INFINITY;
-          for (int j = 0; j < slot; ++j) m = fmaxf(m, a.part_lse[prow0 + j]);
+          for (int j = 0; j < slot; ++j) m = fmaxf(m, a.part_lse[part_lse_at(part_row(prow0 + j, nr))]);
           const float w_own = R.own ? ex2((lse - m) * 1.4426950408889634f) : 0.f;
           float L = w_own;
 #pragma unroll
           for (int x = 0; x < D; ++x) o[x] *= w_own;
           for (int j = 0; j < slot; ++j) {
-            const float wj = ex2((a.part_lse[prow0 + j] - m) * 1.4426950408889634f);
+            const PartRow pj = part_row(prow0 + j, nr);
+            const float wj = ex2((a.part_lse[part_lse_at(pj)] - m) * 1.4426950408889634f);
             L += wj;
-            // 32-byte loads: half the load instructions (each touches one
-            // line per row of the warp) of 16-byte ones
-            const float* src = a.part_o + (prow0 + j) * D;
 #pragma unroll
             for (int x8 = 0; x8 < D / 8; ++x8) {
               float v[8];
-              ld_global_v8(src + 8 * x8, v);
+              ld_global_v8(part_piece(a.part_o, pj, D, x8), v);
 #pragma unroll
               for (int u = 0; u < 8; ++u) o[8 * x8 + u] = fmaf(wj, v[u], o[8 * x8 + u]);
             }
@@ -674,6 +674,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
         // Rows go out through a per-warp staging area so that every global
         // store instruction writes whole 64-byte row pieces of 8 rows.
         const int64_t orow = R.valid ? (MODE == DENSE ? R.t * dm.Hq + R.h : R.prow) : -1;
+        const PartRow prt = part_row(R.valid && MODE != DENSE ? R.prow : 0,
+                                     (int64_t)a.ch.nq * dm.topk);
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t rr[32];
@@ -714,35 +716,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
                 *reinterpret_cast<uint4*>(a.out + o * D + c * 32 + seg * 8) = val;
             }
             __syncwarp();
-          } else {
+          } else if (orow >= 0) {
+            // the row's four 32-byte pieces of these 32 columns, straight
+            // from registers (the interleaved partial layout)
 #pragma unroll
-            for (int rd = 0; rd < 2; ++rd) {  // 32 fp32 columns = 128 bytes per row, 16 rows at a time
-              if ((lane >> 4) == rd) {
+            for (int x = 0; x < 4; ++x) {
+              float v8[8];
 #pragma unroll
-                for (int x = 0; x < 8; ++x)
-                  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                                   stage + (lane & 15) * kStageRow128 + x * 16),
-                               "r"(__float_as_uint(__uint_as_float(rr[4 * x]) * inv_l)),
-                               "r"(__float_as_uint(__uint_as_float(rr[4 * x + 1]) * inv_l)),
-                               "r"(__float_as_uint(__uint_as_float(rr[4 * x + 2]) * inv_l)),
-                               "r"(__float_as_uint(__uint_as_float(rr[4 * x + 3]) * inv_l))
-                               : "memory");
-              }
-              __syncwarp();
-              // 8 lanes per row, 4 rows per instruction
-#pragma unroll
-              for (int it = 0; it < 4; ++it) {
-                const int row = it * 4 + (lane >> 3), seg = lane & 7;
-                const int64_t o = __shfl_sync(0xffffffffu, orow, rd * 16 + row);
-                uint4 val;
-                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                             : "r"(stage + row * kStageRow128 + seg * 16)
-                             : "memory");
-                if (o >= 0)
-                  *reinterpret_cast<uint4*>(a.part_o + o * D + c * 32 + seg * 4) = val;
-              }
-              __syncwarp();
+              for (int u = 0; u < 8; ++u) v8[u] = __uint_as_float(rr[8 * x + u]) * inv_l;
+              st_global_v8(part_piece(a.part_o, prt, D, c * 4 + x), v8);
             }
           }
         }
@@ -750,7 +732,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           if (MODE == DENSE) {
             if (a.lse_out) a.lse_out[R.t * dm.Hq + R.h] = lse;
           } else {
-            a.part_lse[R.prow] = lse;
+            a.part_lse[part_lse_at(prt)] = lse;
           }
         }
       }

@@ -162,9 +162,34 @@ cudaError_t launch_regroup(const Dims& dm, const Chunk& ch, const int32_t* idx, 
 
 // Partial attention results of one pass.
 struct Partials {
-  float* o;    // [T * nq * topk][d], normalised
-  float* lse;  // [T * nq * topk]
+  float* o;    // part_rows(T, nq * topk) rows of d floats, normalised (layout below)
+  float* lse;  // part_rows(T, nq * topk)
 };
+
+// Partial results of a pass are stored interleaved over 32 consecutive
+// tokens. For partial row prow = (t * nq + h_local) * k + slot (nr = nq * k
+// rows per token) the 32-byte piece c of the row (8 floats) sits at piece
+// (tile * (d / 8) + c) * 32 + t % 32 with tile = (t / 32) * nr + prow % nr,
+// and its lse at tile * 32 + t % 32. A warp holding 32 consecutive tokens of
+// one head -- the own-block kernel's merge -- then reads each piece of its
+// rows' partials as one contiguous 1 KB access instead of 32 scattered ones.
+struct PartRow {
+  int64_t tile;
+  int lane;
+};
+__host__ __device__ inline PartRow part_row(int64_t prow, int64_t nr) {
+  const int64_t t = prow / nr;
+  return {(t >> 5) * nr + (prow - t * nr), (int)(t & 31)};
+}
+__host__ __device__ inline float* part_piece(float* o, const PartRow& r, int d, int c) {
+  return o + ((r.tile * (d / 8) + c) * 32 + r.lane) * 8;
+}
+__host__ __device__ inline const float* part_piece(const float* o, const PartRow& r, int d, int c) {
+  return o + ((r.tile * (d / 8) + c) * 32 + r.lane) * 8;
+}
+__host__ __device__ inline int64_t part_lse_at(const PartRow& r) { return r.tile * 32 + r.lane; }
+// Storage rows of a pass: T rounded up to whole 32-token tiles.
+inline size_t part_rows(int64_t T, int64_t nr) { return (size_t)((T + 31) / 32) * 32 * (size_t)nr; }
 
 // Portable SIMT kernels (fp32 or bf16 inputs, any block size).
 cudaError_t launch_history_simt(const Dims& dm, const Chunk& ch, const void* q, const void* k,

@@ -37,11 +37,12 @@ merge_kernel(Dims dm, Chunk ch, const int32_t* __restrict__ idx, const int32_t* 
   const int c = p / dm.B;
   const int32_t* row = idx + (t * dm.Hq + h) * (int64_t)dm.topk;
   const int64_t prow0 = (t * ch.nq + hl) * (int64_t)dm.topk;
+  const int64_t nr = (int64_t)ch.nq * dm.topk;
 
   float m = -INFINITY;
   for (int r = 0; r < dm.topk; ++r) {
     const int e = row[r];
-    if (e >= 0 && e <= c) m = fmaxf(m, part_lse[prow0 + r]);
+    if (e >= 0 && e <= c) m = fmaxf(m, part_lse[part_lse_at(part_row(prow0 + r, nr))]);
   }
   float acc[PL];
 #pragma unroll
@@ -50,9 +51,11 @@ merge_kernel(Dims dm, Chunk ch, const int32_t* __restrict__ idx, const int32_t* 
   for (int r = 0; r < dm.topk; ++r) {
     const int e = row[r];
     if (!(e >= 0 && e <= c)) continue;
-    const float w = expf(part_lse[prow0 + r] - m);
+    const PartRow pr = part_row(prow0 + r, nr);
+    const float w = expf(part_lse[part_lse_at(pr)] - m);
     l += w;
-    const float* src = part_o + (prow0 + r) * D + lane * PL;
+    // lane's PL columns lie inside one 8-column piece
+    const float* src = part_piece(part_o, pr, D, lane * PL / 8) + (lane * PL) % 8;
     if constexpr (PL == 4) {
       const float4 x = *reinterpret_cast<const float4*>(src);
       acc[0] = fmaf(w, x.x, acc[0]);
