@@ -72,13 +72,14 @@ static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr uint32_t kHalf = 128 * 128;  // bytes of one 64-column half of a 128-row tile
 constexpr uint32_t kTile = 2 * kHalf;  // bytes of one 128 x 128 bf16 tile
-constexpr uint32_t kQOff = 0;          // Q[2], one per query half
-constexpr uint32_t kKOff = 2 * kTile;  // K[NS]
+// Q buffers: the (unit, half) loads of a CTA take slots 0, 1, 2, ... in
+// order; slot s uses buffer s % kQBufs. With three buffers for two halves
+// the loader fills the next unit's first half while this unit still computes.
+constexpr int kQBufs = 3;
+constexpr uint32_t kQOff = 0;                // Q[kQBufs]
+constexpr uint32_t kKOff = kQBufs * kTile;   // K[NS]
 constexpr uint32_t kVOff = kKOff + NS * kTile;
-constexpr uint32_t kStageRow = 80;     // bytes per staged row chunk: 64 + 16 pad
-constexpr uint32_t kStageOff = kVOff + NS * kTile;  // epilogue staging, 32 rows per softmax warp
-constexpr uint32_t kStageBytes = 8 * 32 * kStageRow;
-constexpr uint32_t kSmemBytes = kStageOff + kStageBytes + 1024;  // + 1024-byte alignment slack
+constexpr uint32_t kSmemBytes = kVOff + NS * kTile + 1024;  // + 1024-byte alignment slack
 constexpr uint32_t kTmemCols = 512;    // S[0] 0, S[1] 128, O[0] 256, O[1] 384
 constexpr uint32_t kOCol = 256;
 constexpr uint32_t kIdescQK = idesc_bf16(TM, TN, false, false);  // Q, K both K-major
@@ -87,7 +88,8 @@ constexpr float kRescaleLog2 = 8.f;
 
 struct Shared {
   // per query half h
-  uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_free[2];
+  uint64_t q_full[kQBufs], q_empty[kQBufs];
+  uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
   uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
   uint64_t drain[2];
   uint32_t tmem_base;
@@ -282,9 +284,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
   const uint32_t sQ = sbase + kQOff, sK = sbase + kKOff, sV = sbase + kVOff;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kQBufs; ++i) {
       mbar_init(&sh.q_full[i], kLoaderThreads);
       mbar_init(&sh.q_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&sh.s_full[i], 1);
       mbar_init(&sh.p_full[i], 128);
       mbar_init(&sh.o_full[i], 1);
@@ -360,11 +364,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
         uint32_t gk = 0;  // KV tiles streamed before this unit
         uint32_t kh = 0;  // KV tiles of this half before this unit
         uint32_t uh = 0;  // units with this half non-empty before this one
+        uint32_t qs = 0;  // Q slots (loads of either half) before this unit
         bool ok = true;
         for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
           const Tile T = get_tile<MODE>(a, t);
           if (T.skip) continue;
           const int nh = T.n[h];
+          const uint32_t qslot = qs + (h == 1 && T.n[0] > 0 ? 1u : 0u);
+          const uint32_t qb = qslot % kQBufs;
+          qs += (T.n[0] > 0 ? 1u : 0u) + (T.n[1] > 0 ? 1u : 0u);
           for (int j = 0; ok && j < T.n_kv; ++j) {
             const uint32_t gg = gk + j, st = gg % NS;
             // Both issuers wait for every tile, also one they skip, before
@@ -374,17 +382,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
             if (j < nh) {
               // S[h] = Q_h K(j)^T; S[h] holds P(j - 1) until PV(j - 1), which
               // this thread issued before
-              if (j == 0 && !(ok = mbar_wait(&sh.q_full[h], uh & 1, abort, status))) break;
+              if (j == 0 &&
+                  !(ok = mbar_wait(&sh.q_full[qb], (qslot / kQBufs) & 1, abort, status)))
+                break;
               fence_after_sync();
 #pragma unroll
               for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-                const uint64_t ad = desc_sw128(sQ + h * kTile + off, 16, 1024);
+                const uint64_t ad = desc_sw128(sQ + qb * kTile + off, 16, 1024);
                 const uint64_t bd = desc_sw128(sK + st * kTile + off, 16, 1024);
                 mma_ss(tmem + h * 128, ad, bd, kIdescQK, kk > 0 ? 1u : 0u);
               }
               commit(&sh.s_full[h]);
-              if (j == nh - 1) commit(&sh.q_empty[h]);
+              if (j == nh - 1) commit(&sh.q_empty[qb]);
             }
             commit(&sh.k_empty[st]);
             if (j < nh) {
@@ -419,38 +429,71 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
       }
     } else {
       // ================= Q loader, warp 3 =================
+      // The row ids of a unit (tile table -> list offset -> pairs: three
+      // dependent global loads in the history kernel) are fetched one unit
+      // ahead, while the current unit computes, so a freed Q buffer waits
+      // only for its copies.
+      constexpr int RPL = TM / kLoaderThreads;  // rows per lane and half
       const int tl = lane;
-      uint32_t ul[2] = {0, 0};
+      uint32_t qs = 0;  // Q slots loaded so far
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+      auto next_unit = [&](int t) {
+        for (; t < n_tiles; t += gridDim.x)
+          if (!get_tile<MODE>(a, t).skip) break;
+        return t;
+      };
+      // row ids (t * Hq + h < 2^31, checked on the host) of both halves of
+      // unit t, -1 where a row is empty; bit h of the result: half h reads
+      auto fetch_rows = [&](int t, int32_t (&qr)[2][RPL]) {
         const Tile T = get_tile<MODE>(a, t);
-        if (T.skip) continue;
+        int mask = 0;
+#pragma unroll
         for (int h = 0; h < 2; ++h) {
-          if (T.n[h] == 0) continue;
-          if (ul[h] > 0) {
-            ok = mbar_wait(&sh.q_empty[h], (ul[h] - 1) & 1, abort, status);
+          const Tile U = half_view<MODE>(T, h);
+          if (T.n[h] > 0) mask |= 1 << h;
+#pragma unroll
+          for (int hr = 0; hr < RPL; ++hr) {
+            int64_t qrow = -1;
+            if (T.n[h] == 0 || !q_row_of<MODE>(a, U, tl + hr * kLoaderThreads, qrow)) qrow = -1;
+            qr[h][hr] = (int32_t)qrow;
+          }
+        }
+        return mask;
+      };
+      int t = next_unit(blockIdx.x);
+      int32_t qr[2][RPL];
+      int mask = t < n_tiles ? fetch_rows(t, qr) : 0;
+      while (ok && t < n_tiles) {
+        for (int h = 0; h < 2; ++h) {
+          if (!(mask >> h & 1)) continue;
+          const uint32_t qb = qs % kQBufs;
+          if (qs >= (uint32_t)kQBufs) {
+            ok = mbar_wait(&sh.q_empty[qb], (qs / kQBufs - 1) & 1, abort, status);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           }
-          const Tile U = half_view<MODE>(T, h);
-  #pragma unroll
-          for (int hr = 0; hr < TM / kLoaderThreads; ++hr) {
+#pragma unroll
+          for (int hr = 0; hr < RPL; ++hr) {
             const int rr = tl + hr * kLoaderThreads;
-            int64_t qrow = 0;
-            const bool has = q_row_of<MODE>(a, U, rr, qrow);
-            const __nv_bfloat16* src = a.q + (has ? qrow : 0) * (int64_t)D;
-  #pragma unroll
+            const bool has = qr[h][hr] >= 0;
+            const __nv_bfloat16* src = a.q + (has ? (int64_t)qr[h][hr] : 0) * (int64_t)D;
+#pragma unroll
             for (int c16 = 0; c16 < 16; ++c16) {
-              const uint32_t dst = sQ + h * kTile + (c16 >> 3) * kHalf + rr * 128 +
+              const uint32_t dst = sQ + qb * kTile + (c16 >> 3) * kHalf + rr * 128 +
                                    ((((uint32_t)c16 & 7u) ^ ((uint32_t)rr & 7u)) << 4);
               cp_async16(dst, src + c16 * 8, has ? 16u : 0u);
             }
           }
           cp_async_wait_all();
           fence_proxy_async_smem();
-          mbar_arrive(&sh.q_full[h]);
-          ++ul[h];
+          mbar_arrive(&sh.q_full[qb]);
+          ++qs;
         }
+        if (!ok) break;
+        // the next unit's row ids, while this unit computes
+        t = next_unit(t + gridDim.x);
+        mask = t < n_tiles ? fetch_rows(t, qr) : 0;
       }
+      cp_async_wait_all();
     }
   } else {
     regs_inc();
@@ -462,7 +505,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
     const uint32_t tS = tmem + hh * 128 + lane_addr;
     const uint32_t tO = tmem + kOCol + hh * 128 + lane_addr;
     const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;  // softmax scale, base 2
-    const uint32_t stage = sbase + kStageOff + (warp - 4) * 32 * kStageRow;
     uint32_t kc = 0, uc = 0;
     int base[2] = {0, 0};  // KV tiles each half processed in earlier units
     volatile int* exp_cnt = sh.exp_cnt;
@@ -606,13 +648,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
         const int64_t prow0 = R.valid ? R.prow : 0;
         const int64_t orow = R.valid ? R.t * dm.Hq + R.h : -1;
         float o[D];
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t rr[32];
-          tmem_ld32(tO + c * 32, rr);
+        {
+          // all four loads in flight, then one wait
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          tmem_ld32(tO, r0);
+          tmem_ld32(tO + 32, r1);
+          tmem_ld32(tO + 64, r2);
+          tmem_ld32(tO + 96, r3);
           tmem_wait_ld();
 #pragma unroll
-          for (int x = 0; x < 32; ++x) o[c * 32 + x] = __uint_as_float(rr[x]) * inv_l;
+          for (int x = 0; x < 32; ++x) {
+            o[x] = __uint_as_float(r0[x]) * inv_l;
+            o[32 + x] = __uint_as_float(r1[x]) * inv_l;
+            o[64 + x] = __uint_as_float(r2[x]) * inv_l;
+            o[96 + x] = __uint_as_float(r3[x]) * inv_l;
+          }
         }
         // O[h] is in registers: the next unit's PV may overwrite it
         fence_before_sync();
@@ -642,89 +692,61 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           for (int x = 0; x < D; ++x) o[x] *= inv;
           if (a.lse_out) a.lse_out[orow] = m + logf(L);
         }
-        // the bf16 row leaves through the staging area in 64-byte pieces
+        // the bf16 row leaves straight from registers in 32-byte pieces
+        if (orow >= 0) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+          for (int x16 = 0; x16 < D / 16; ++x16) {
+            uint32_t w[8];
 #pragma unroll
-          for (int x = 0; x < 4; ++x)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                             stage + lane * kStageRow + x * 16),
-                         "r"(pack_bf16x2(o[c * 32 + 8 * x], o[c * 32 + 8 * x + 1])),
-                         "r"(pack_bf16x2(o[c * 32 + 8 * x + 2], o[c * 32 + 8 * x + 3])),
-                         "r"(pack_bf16x2(o[c * 32 + 8 * x + 4], o[c * 32 + 8 * x + 5])),
-                         "r"(pack_bf16x2(o[c * 32 + 8 * x + 6], o[c * 32 + 8 * x + 7]))
-                         : "memory");
-          __syncwarp();
-          // 64 bytes per row chunk: 4 lanes per row, 8 rows per instruction
-#pragma unroll
-          for (int it = 0; it < 4; ++it) {
-            const int row = it * 8 + (lane >> 2), seg = lane & 3;
-            const int64_t orr = __shfl_sync(0xffffffffu, orow, row);
-            uint4 val;
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                         : "r"(stage + row * kStageRow + seg * 16)
-                         : "memory");
-            if (orr >= 0)
-              *reinterpret_cast<uint4*>(a.out + orr * D + c * 32 + seg * 8) = val;
+            for (int u = 0; u < 8; ++u) w[u] = pack_bf16x2(o[16 * x16 + 2 * u], o[16 * x16 + 2 * u + 1]);
+            st_global_v8_b32(a.out + orow * D + 16 * x16, w);
           }
-          __syncwarp();
         }
       } else {
-        // Rows go out through a per-warp staging area so that every global
-        // store instruction writes whole 64-byte row pieces of 8 rows.
+        // Each thread writes its own row in 32-byte pieces (a warp store
+        // covers 32 rows; every 32-byte sector is written whole).
         const int64_t orow = R.valid ? (MODE == DENSE ? R.t * dm.Hq + R.h : R.prow) : -1;
         const PartRow prt = part_row(R.valid && MODE != DENSE ? R.prow : 0,
                                      (int64_t)a.ch.nq * dm.topk);
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t rr[32];
-          tmem_ld32(tO + c * 32, rr);
+        uint32_t ro[D];
+        {
+          // all four loads in flight, then one wait; O[h] is then in
+          // registers and the next unit's PV may overwrite it
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          tmem_ld32(tO, r0);
+          tmem_ld32(tO + 32, r1);
+          tmem_ld32(tO + 64, r2);
+          tmem_ld32(tO + 96, r3);
           tmem_wait_ld();
-          if (c == D / 32 - 1) {
-            // O[h] is in registers: the next unit's PV may overwrite it
-            fence_before_sync();
-            mbar_arrive(&sh.o_free[hh]);
+          fence_before_sync();
+          mbar_arrive(&sh.o_free[hh]);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            ro[x] = r0[x];
+            ro[32 + x] = r1[x];
+            ro[64 + x] = r2[x];
+            ro[96 + x] = r3[x];
           }
+        }
+        if (orow >= 0) {
           if (MODE == DENSE) {
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              const uint32_t w0 = pack_bf16x2(__uint_as_float(rr[8 * x]) * inv_l,
-                                              __uint_as_float(rr[8 * x + 1]) * inv_l);
-              const uint32_t w1 = pack_bf16x2(__uint_as_float(rr[8 * x + 2]) * inv_l,
-                                              __uint_as_float(rr[8 * x + 3]) * inv_l);
-              const uint32_t w2 = pack_bf16x2(__uint_as_float(rr[8 * x + 4]) * inv_l,
-                                              __uint_as_float(rr[8 * x + 5]) * inv_l);
-              const uint32_t w3 = pack_bf16x2(__uint_as_float(rr[8 * x + 6]) * inv_l,
-                                              __uint_as_float(rr[8 * x + 7]) * inv_l);
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                               stage + lane * kStageRow + x * 16),
-                           "r"(w0), "r"(w1), "r"(w2), "r"(w3)
-                           : "memory");
-            }
-            __syncwarp();
+            for (int x16 = 0; x16 < D / 16; ++x16) {
+              uint32_t w[8];
 #pragma unroll
-            for (int it = 0; it < 4; ++it) {
-              const int row = it * 8 + (lane >> 2), seg = lane & 3;
-              const int64_t o = __shfl_sync(0xffffffffu, orow, row);
-              uint4 val;
-              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                           : "r"(stage + row * kStageRow + seg * 16)
-                           : "memory");
-              if (o >= 0)
-                *reinterpret_cast<uint4*>(a.out + o * D + c * 32 + seg * 8) = val;
+              for (int u = 0; u < 8; ++u)
+                w[u] = pack_bf16x2(__uint_as_float(ro[16 * x16 + 2 * u]) * inv_l,
+                                   __uint_as_float(ro[16 * x16 + 2 * u + 1]) * inv_l);
+              st_global_v8_b32(a.out + orow * D + 16 * x16, w);
             }
-            __syncwarp();
-          } else if (orow >= 0) {
-            // the row's four 32-byte pieces of these 32 columns, straight
-            // from registers (the interleaved partial layout)
+          } else {
+            // the row's 32-byte pieces (the interleaved partial layout)
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
+            for (int x8 = 0; x8 < D / 8; ++x8) {
               float v8[8];
 #pragma unroll
-              for (int u = 0; u < 8; ++u) v8[u] = __uint_as_float(rr[8 * x + u]) * inv_l;
-              st_global_v8(part_piece(a.part_o, prt, D, c * 4 + x), v8);
+              for (int u = 0; u < 8; ++u) v8[u] = __uint_as_float(ro[8 * x8 + u]) * inv_l;
+              st_global_v8(part_piece(a.part_o, prt, D, x8), v8);
             }
           }
         }
