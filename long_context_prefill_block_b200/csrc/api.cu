@@ -126,7 +126,7 @@ Layout plan(const Dims& dm, bool own_idx) {
   L.pairs = take(sizeof(int32_t) * max_pairs);
   L.tiles = take(sizeof(int2) * L.max_tiles);
   const size_t prows = part_rows(dm.T, (int64_t)L.ng * grp * dm.topk);
-  L.part_o = take(sizeof(float) * prows * dm.d);
+  L.part_o = take((dm.dtype == kBF16 ? 2 : 4) * prows * dm.d);
   L.part_lse = take(sizeof(float) * prows);
   L.total = off;
   return L;
@@ -203,7 +203,7 @@ moba_status forward_impl(const moba_params* p, const void* q, const void* k, con
   rg.tile_off = reinterpret_cast<int32_t*>(base + L.tile_off);
   rg.pairs = reinterpret_cast<int32_t*>(base + L.pairs);
   rg.tiles = reinterpret_cast<int2*>(base + L.tiles);
-  Partials pt{reinterpret_cast<float*>(base + L.part_o), reinterpret_cast<float*>(base + L.part_lse)};
+  Partials pt{base + L.part_o, reinterpret_cast<float*>(base + L.part_lse)};
   for (int g0 = 0; g0 < dm.Hkv; g0 += L.ng) {
     Chunk ch;
     ch.g0 = g0;

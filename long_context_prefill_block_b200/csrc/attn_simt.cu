@@ -32,7 +32,7 @@ attn_simt(Dims dm, Chunk ch, const T* __restrict__ q, const T* __restrict__ k,
           const T* __restrict__ v, const int32_t* __restrict__ cu,
           const int32_t* __restrict__ list_off, const int32_t* __restrict__ pairs,
           const int2* __restrict__ tiles, const int32_t* __restrict__ tile_count,
-          const int32_t* __restrict__ idx, float* __restrict__ part_o,
+          const int32_t* __restrict__ idx, void* __restrict__ part_o,
           float* __restrict__ part_lse, T* __restrict__ out, float* __restrict__ lse_out) {
   __shared__ __align__(16) float ks[kKC][D + 4];
   __shared__ __align__(16) float vs[kKC][D + 4];
@@ -194,12 +194,13 @@ attn_simt(Dims dm, Chunk ch, const T* __restrict__ q, const T* __restrict__ k,
     if (lse_out && part == 0) lse_out[t * dm.Hq + h] = lse;
   } else {
     const PartRow pr = part_row(prow, (int64_t)ch.nq * dm.topk);
+    constexpr int PE = 32 / (int)sizeof(T);  // values per 32-byte piece
 #pragma unroll
     for (int j = 0; j < NG; ++j) {
-      const int x0 = part * 4 + 16 * j;  // four columns inside one 8-column piece
-      *reinterpret_cast<float4*>(part_piece(part_o, pr, D, x0 / 8) + x0 % 8) =
-          make_float4(o[j * 4] * inv_l, o[j * 4 + 1] * inv_l, o[j * 4 + 2] * inv_l,
-                      o[j * 4 + 3] * inv_l);
+      const int x0 = part * 4 + 16 * j;  // four columns inside one piece
+      T* dst = part_piece<T>(part_o, pr, D, x0 / PE) + x0 % PE;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) dst[u] = from_f32<T>(o[j * 4 + u] * inv_l);
     }
     if (part == 0) part_lse[part_lse_at(pr)] = lse;
   }

@@ -111,7 +111,7 @@ struct Args {
   // CUR
   const int32_t* idx;
   // outputs
-  float* part_o;
+  void* part_o;  // bf16 partial rows, interleaved layout
   float* part_lse;
   __nv_bfloat16* out;
   float* lse_out;
@@ -680,11 +680,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
             const float wj = ex2((a.part_lse[part_lse_at(pj)] - m) * 1.4426950408889634f);
             L += wj;
 #pragma unroll
-            for (int x8 = 0; x8 < D / 8; ++x8) {
-              float v[8];
-              ld_global_v8(part_piece(a.part_o, pj, D, x8), v);
+            for (int x16 = 0; x16 < D / 16; ++x16) {
+              uint32_t v[8];  // 16 bf16 values
+              ld_global_v8_b32(part_piece<__nv_bfloat16>(a.part_o, pj, D, x16), v);
 #pragma unroll
-              for (int u = 0; u < 8; ++u) o[8 * x8 + u] = fmaf(wj, v[u], o[8 * x8 + u]);
+              for (int u = 0; u < 8; ++u) {
+                o[16 * x16 + 2 * u] = fmaf(wj, __uint_as_float(v[u] << 16), o[16 * x16 + 2 * u]);
+                o[16 * x16 + 2 * u + 1] =
+                    fmaf(wj, __uint_as_float(v[u] & 0xffff0000u), o[16 * x16 + 2 * u + 1]);
+              }
             }
           }
           const float inv = 1.f / L;
@@ -740,13 +744,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
               st_global_v8_b32(a.out + orow * D + 16 * x16, w);
             }
           } else {
-            // the row's 32-byte pieces (the interleaved partial layout)
+            // the row's 32-byte pieces of 16 bf16 (the interleaved partial layout)
 #pragma unroll
-            for (int x8 = 0; x8 < D / 8; ++x8) {
-              float v8[8];
+            for (int x16 = 0; x16 < D / 16; ++x16) {
+              uint32_t w[8];
 #pragma unroll
-              for (int u = 0; u < 8; ++u) v8[u] = __uint_as_float(ro[8 * x8 + u]) * inv_l;
-              st_global_v8(part_piece(a.part_o, prt, D, x8), v8);
+              for (int u = 0; u < 8; ++u)
+                w[u] = pack_bf16x2(__uint_as_float(ro[16 * x16 + 2 * u]) * inv_l,
+                                   __uint_as_float(ro[16 * x16 + 2 * u + 1]) * inv_l);
+              st_global_v8_b32(part_piece<__nv_bfloat16>(a.part_o, prt, D, x16), w);
             }
           }
         }

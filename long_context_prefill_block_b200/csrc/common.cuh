@@ -162,17 +162,22 @@ cudaError_t launch_regroup(const Dims& dm, const Chunk& ch, const int32_t* idx, 
 
 // Partial attention results of one pass.
 struct Partials {
-  float* o;    // part_rows(T, nq * topk) rows of d floats, normalised (layout below)
+  void* o;     // part_rows(T, nq * topk) rows of d values in the input dtype (layout below)
   float* lse;  // part_rows(T, nq * topk)
 };
 
+// A partial result o_j = u_j / l_j (normalised, so |o_j| <= max |v|) is
+// stored in the input dtype -- bf16 for bf16 inputs, as merge-state kernels
+// commonly keep it -- and merged in fp32; its lse stays fp32.
+//
 // Partial results of a pass are stored interleaved over 32 consecutive
 // tokens. For partial row prow = (t * nq + h_local) * k + slot (nr = nq * k
-// rows per token) the 32-byte piece c of the row (8 floats) sits at piece
-// (tile * (d / 8) + c) * 32 + t % 32 with tile = (t / 32) * nr + prow % nr,
-// and its lse at tile * 32 + t % 32. A warp holding 32 consecutive tokens of
-// one head -- the own-block kernel's merge -- then reads each piece of its
-// rows' partials as one contiguous 1 KB access instead of 32 scattered ones.
+// rows per token) the 32-byte piece c of the row sits at piece
+// (tile * npc + c) * 32 + t % 32 (npc = the row's 32-byte pieces) with
+// tile = (t / 32) * nr + prow % nr, and its lse at tile * 32 + t % 32. A
+// warp holding 32 consecutive tokens of one head -- the own-block kernel's
+// merge -- then reads each piece of its rows' partials as one contiguous
+// 1 KB access instead of 32 scattered ones.
 struct PartRow {
   int64_t tile;
   int lane;
@@ -181,11 +186,15 @@ __host__ __device__ inline PartRow part_row(int64_t prow, int64_t nr) {
   const int64_t t = prow / nr;
   return {(t >> 5) * nr + (prow - t * nr), (int)(t & 31)};
 }
-__host__ __device__ inline float* part_piece(float* o, const PartRow& r, int d, int c) {
-  return o + ((r.tile * (d / 8) + c) * 32 + r.lane) * 8;
+template <typename P>
+__host__ __device__ inline P* part_piece(void* o, const PartRow& r, int d, int c) {
+  const int npc = d * (int)sizeof(P) / 32;
+  return reinterpret_cast<P*>(static_cast<char*>(o) + ((r.tile * npc + c) * 32 + r.lane) * 32);
 }
-__host__ __device__ inline const float* part_piece(const float* o, const PartRow& r, int d, int c) {
-  return o + ((r.tile * (d / 8) + c) * 32 + r.lane) * 8;
+template <typename P>
+__host__ __device__ inline const P* part_piece(const void* o, const PartRow& r, int d, int c) {
+  const int npc = d * (int)sizeof(P) / 32;
+  return reinterpret_cast<const P*>(static_cast<const char*>(o) + ((r.tile * npc + c) * 32 + r.lane) * 32);
 }
 __host__ __device__ inline int64_t part_lse_at(const PartRow& r) { return r.tile * 32 + r.lane; }
 // Storage rows of a pass: T rounded up to whole 32-token tiles.

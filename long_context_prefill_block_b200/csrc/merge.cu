@@ -23,7 +23,7 @@ constexpr int kWarps = 4;
 template <typename T, int D>
 __global__ void __launch_bounds__(kWarps * 32)
 merge_kernel(Dims dm, Chunk ch, const int32_t* __restrict__ idx, const int32_t* __restrict__ cu,
-             const float* __restrict__ part_o, const float* __restrict__ part_lse,
+             const void* __restrict__ part_o, const float* __restrict__ part_lse,
              T* __restrict__ out, float* __restrict__ lse_out) {
   constexpr int PL = D / 32;  // columns per lane
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -54,18 +54,11 @@ merge_kernel(Dims dm, Chunk ch, const int32_t* __restrict__ idx, const int32_t* 
     const PartRow pr = part_row(prow0 + r, nr);
     const float w = expf(part_lse[part_lse_at(pr)] - m);
     l += w;
-    // lane's PL columns lie inside one 8-column piece
-    const float* src = part_piece(part_o, pr, D, lane * PL / 8) + (lane * PL) % 8;
-    if constexpr (PL == 4) {
-      const float4 x = *reinterpret_cast<const float4*>(src);
-      acc[0] = fmaf(w, x.x, acc[0]);
-      acc[1] = fmaf(w, x.y, acc[1]);
-      acc[2] = fmaf(w, x.z, acc[2]);
-      acc[3] = fmaf(w, x.w, acc[3]);
-    } else {
+    // lane's PL columns lie inside one 32-byte piece (partials in T)
+    constexpr int PE = 32 / (int)sizeof(T);
+    const T* src = part_piece<T>(part_o, pr, D, lane * PL / PE) + (lane * PL) % PE;
 #pragma unroll
-      for (int u = 0; u < PL; ++u) acc[u] = fmaf(w, src[u], acc[u]);
-    }
+    for (int u = 0; u < PL; ++u) acc[u] = fmaf(w, to_f32(src[u]), acc[u]);
   }
   const float inv_l = 1.f / l;
   T* dst = out + (t * dm.Hq + h) * (int64_t)D + lane * PL;
