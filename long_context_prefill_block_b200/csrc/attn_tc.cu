@@ -579,16 +579,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           l_i *= ex2(m_i - m_new);
           m_i = m_new;
         }
-        // CUR / DENSE: the two halves take turns on the exponential unit:
-        // half 1 exponentiates KV tile j after half 0 has, half 0 tile j
-        // after half 1 has done tile j - 1. In anti-phase, one half's PV and
-        // next QK^T run while the other half exponentiates. (HIST units are
-        // only B / 128 KV tiles long and run faster without the turns: one
+        // DENSE: the two halves take turns on the exponential unit: half 1
+        // exponentiates KV tile j after half 0 has, half 0 tile j after half
+        // 1 has done tile j - 1. In anti-phase, one half's PV and next QK^T
+        // run while the other half exponentiates. (HIST and CUR units are
+        // only a few KV tiles long and run faster without the turns: one
         // warp per SM sub-partition reaches only about half the exponential
         // rate of two.)
         // Counts only grow, so a half that runs ahead into its next unit
         // cannot be mistaken for the turn being waited for.
-        if (MODE != HIST && (hh == 0 ? (j >= 1 && j - 1 < T0.n[1]) : (j < T0.n[0]))) {
+        if (MODE == DENSE && (hh == 0 ? (j >= 1 && j - 1 < T0.n[1]) : (j < T0.n[0]))) {
           const int need_cnt = 4 * (hh == 0 ? b1 + j : b0 + j + 1);
           const long long t0 = clock64();
           while (exp_cnt[hh ^ 1] < need_cnt) {
