@@ -366,8 +366,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
         uint32_t uh = 0;  // units with this half non-empty before this one
         uint32_t qs = 0;  // Q slots (loads of either half) before this unit
         bool ok = true;
+        Tile Tnext = (int)blockIdx.x < n_tiles ? get_tile<MODE>(a, blockIdx.x) : Tile{};
         for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-          const Tile T = get_tile<MODE>(a, t);
+          const Tile T = Tnext;  // read one unit ahead
+          if (t + (int)gridDim.x < n_tiles) Tnext = get_tile<MODE>(a, t + gridDim.x);
           if (T.skip) continue;
           const int nh = T.n[h];
           const uint32_t qslot = qs + (h == 1 && T.n[0] > 0 ? 1u : 0u);
@@ -509,8 +511,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
     int base[2] = {0, 0};  // KV tiles each half processed in earlier units
     volatile int* exp_cnt = sh.exp_cnt;
     bool ok = true;
+    // the unit's description is read one unit ahead: its global loads (tile
+    // table, list offsets, sequence bounds) resolve while this unit runs
+    Tile Tnext = (int)blockIdx.x < n_tiles ? get_tile<MODE>(a, blockIdx.x) : Tile{};
     for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-      const Tile T0 = get_tile<MODE>(a, t);
+      const Tile T0 = Tnext;
+      if (t + (int)gridDim.x < n_tiles) Tnext = get_tile<MODE>(a, t + gridDim.x);
       if (T0.skip) continue;
       const int b0 = base[0], b1 = base[1];
       base[0] += T0.n[0];
