@@ -635,11 +635,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
       }
       if (!ok) break;
       // ---- epilogue: wait for the half's last PV, normalise, write
+      const float inv_l = 1.f / l_i;
+      const float lse = (m_i + log2f(l_i)) * 0.6931471805599453f;
+      // CUR: the merge weights need only the lse values, not the last PV:
+      // they are read (and the weights formed) while the PV runs
+      constexpr int kPreLse = 4;
+      float wpre[kPreLse];
+      float m_all = -INFINITY, L_all = 0.f, w_own = 0.f;
+      if (MODE == CUR && R.valid) {
+        const int64_t nr = (int64_t)a.ch.nq * dm.topk;
+        float lj[kPreLse];
+#pragma unroll
+        for (int j = 0; j < kPreLse; ++j)
+          lj[j] = j < R.nhist ? a.part_lse[part_lse_at(part_row(R.prow + j, nr))] : -INFINITY;
+        m_all = R.own ? lse : -INFINITY;
+#pragma unroll
+        for (int j = 0; j < kPreLse; ++j) m_all = fmaxf(m_all, lj[j]);
+        for (int j = kPreLse; j < R.nhist; ++j)
+          m_all = fmaxf(m_all, a.part_lse[part_lse_at(part_row(R.prow + j, nr))]);
+        w_own = R.own ? ex2((lse - m_all) * 1.4426950408889634f) : 0.f;
+        L_all = w_own;
+#pragma unroll
+        for (int j = 0; j < kPreLse; ++j) {
+          wpre[j] = j < R.nhist ? ex2((lj[j] - m_all) * 1.4426950408889634f) : 0.f;
+          L_all += wpre[j];
+        }
+        for (int j = kPreLse; j < R.nhist; ++j)
+          L_all += ex2((a.part_lse[part_lse_at(part_row(R.prow + j, nr))] - m_all) *
+                       1.4426950408889634f);
+      }
       ok = mbar_wait(&sh.o_full[hh], uc & 1, abort, status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       fence_after_sync();
-      const float inv_l = 1.f / l_i;
-      const float lse = (m_i + log2f(l_i)) * 0.6931471805599453f;
       if (MODE == CUR) {
         // Own block done: merge with this row's history partials right here
         // (eq. 7-8 written with lse: w_j = exp(lse_j - m), o = sum_j w_j o_j /
@@ -675,16 +702,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
         mbar_arrive(&sh.o_free[hh]);
         if (R.valid) {
           const int64_t nr = (int64_t)a.ch.nq * dm.topk;
-          float m = R.own ? lse : -INFINITY;
-          for (int j = 0; j < slot; ++j) m = fmaxf(m, a.part_lse[part_lse_at(part_row(prow0 + j, nr))]);
-          const float w_own = R.own ? ex2((lse - m) * 1.4426950408889634f) : 0.f;
-          float L = w_own;
+          const float m = m_all, L = L_all;
 #pragma unroll
           for (int x = 0; x < D; ++x) o[x] *= w_own;
           for (int j = 0; j < slot; ++j) {
             const PartRow pj = part_row(prow0 + j, nr);
-            const float wj = ex2((a.part_lse[part_lse_at(pj)] - m) * 1.4426950408889634f);
-            L += wj;
+            float wj = 0.f;
+#pragma unroll
+            for (int q = 0; q < kPreLse; ++q)
+              if (q == j) wj = wpre[q];
+            if (j >= kPreLse) wj = ex2((a.part_lse[part_lse_at(pj)] - m) * 1.4426950408889634f);
 #pragma unroll
             for (int x16 = 0; x16 < D / 16; ++x16) {
               uint32_t v[8];  // 16 bf16 values
