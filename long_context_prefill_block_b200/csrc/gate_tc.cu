@@ -135,7 +135,9 @@ __device__ __forceinline__ int next_valid(const GateArgs& a, const int32_t* cu, 
   }
 }
 
-template <int KM>
+// PFX: the own block is scored by its prefix mean (compiled separately, so
+// the forced-own-block kernel carries none of that code)
+template <int KM, bool PFX>
 __global__ void __launch_bounds__(kThreads, KM <= 4 ? 3 : 1)
 gate_tc_kernel(const __grid_constant__ CUtensorMap tmq, const GateArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -362,7 +364,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmq, const GateArgs a) {
       // the own block: forced, or (prefix mean) in unless k earlier blocks
       // score at least as high; it loses ties, being the highest index
       bool own_in = true;
-      if (dm.prefix && c >= dm.topk) {
+      if (PFX && c >= dm.topk) {
         float kth = -INFINITY, so = 0.f;
 #pragma unroll
         for (int j = 0; j < KM; ++j)
@@ -414,10 +416,10 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmq, const GateArgs a) {
 
 constexpr int kMaxSmem = 232448;  // 227 KB per CTA
 
-// CTAs of gate_tc_kernel<KM> per SM at `smem` bytes of dynamic shared
+// CTAs of gate_tc_kernel<KM, PFX> per SM at `smem` bytes of dynamic shared
 // memory, bounded by registers and shared memory (counted here from the
 // kernel's attributes, asked once per device and remembered).
-template <int KM>
+template <int KM, bool PFX>
 cudaError_t occupancy(int* n, size_t smem) {
   static std::mutex mu;
   static cudaFuncAttributes attrs[kMaxDevices];
@@ -428,9 +430,10 @@ cudaError_t occupancy(int* n, size_t smem) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
   if (!have[dev]) {
-    if ((e = cudaFuncGetAttributes(&attrs[dev], gate_tc_kernel<KM>))) return e;
+    if ((e = cudaFuncGetAttributes(&attrs[dev], gate_tc_kernel<KM, PFX>))) return e;
     // allow all the dynamic shared memory the static part leaves
-    if ((e = cudaFuncSetAttribute(gate_tc_kernel<KM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if ((e = cudaFuncSetAttribute(gate_tc_kernel<KM, PFX>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   kMaxSmem - (int)attrs[dev].sharedSizeBytes)))
       return e;
     have[dev] = true;
@@ -449,9 +452,9 @@ cudaError_t occupancy(int* n, size_t smem) {
   return cudaSuccess;
 }
 
-template <int KM>
+template <int KM, bool PFX>
 cudaError_t run(const CUtensorMap& mq, const GateArgs& a, size_t smem, int grid, cudaStream_t st) {
-  gate_tc_kernel<KM><<<grid, kThreads, smem, st>>>(mq, a);
+  gate_tc_kernel<KM, PFX><<<grid, kThreads, smem, st>>>(mq, a);
   return cudaGetLastError();
 }
 
@@ -461,8 +464,10 @@ bool gate_tc_supported(const Dims& dm) {
   return dm.dtype == kBF16 && dm.d == 128 && dm.nb <= kMaxBlocks && dm.topk <= 33;
 }
 
-cudaError_t launch_gate_tc(const Dims& dm, const void* q, const float* kbar, const float* own,
-                           const int32_t* cu, int32_t* idx, int* status, cudaStream_t st) {
+namespace {
+template <bool PFX>
+cudaError_t launch_impl(const Dims& dm, const void* q, const float* kbar, const float* own,
+                        const int32_t* cu, int32_t* idx, int* status, cudaStream_t st) {
   if (dm.batch == 0 || dm.max_seqlen == 0) return cudaSuccess;
   GateArgs a{};
   a.dm = dm;
@@ -497,12 +502,12 @@ cudaError_t launch_gate_tc(const Dims& dm, const void* q, const float* kbar, con
     int n = 0;
     cudaError_t e2;
     switch (need_km) {
-      case 1: e2 = occupancy<1>(&n, smem); break;
-      case 2: e2 = occupancy<2>(&n, smem); break;
-      case 4: e2 = occupancy<4>(&n, smem); break;
-      case 8: e2 = occupancy<8>(&n, smem); break;
-      case 16: e2 = occupancy<16>(&n, smem); break;
-      default: e2 = occupancy<32>(&n, smem); break;
+      case 1: e2 = occupancy<1, PFX>(&n, smem); break;
+      case 2: e2 = occupancy<2, PFX>(&n, smem); break;
+      case 4: e2 = occupancy<4, PFX>(&n, smem); break;
+      case 8: e2 = occupancy<8, PFX>(&n, smem); break;
+      case 16: e2 = occupancy<16, PFX>(&n, smem); break;
+      default: e2 = occupancy<32, PFX>(&n, smem); break;
     }
     if (e2 != cudaSuccess) return 0;
     if (n > (int)(512 / cols)) n = (int)(512 / cols);
@@ -525,12 +530,20 @@ cudaError_t launch_gate_tc(const Dims& dm, const void* q, const float* kbar, con
   CUtensorMap mq;
   cudaError_t e = make_head_map(&mq, q, dm.T, dm.Hq, kTileRows);
   if (e != cudaSuccess) return e;
-  if (need <= 1) return run<1>(mq, a, smem, grid, st);
-  if (need <= 2) return run<2>(mq, a, smem, grid, st);
-  if (need <= 4) return run<4>(mq, a, smem, grid, st);
-  if (need <= 8) return run<8>(mq, a, smem, grid, st);
-  if (need <= 16) return run<16>(mq, a, smem, grid, st);
-  return run<32>(mq, a, smem, grid, st);
+  if (need <= 1) return run<1, PFX>(mq, a, smem, grid, st);
+  if (need <= 2) return run<2, PFX>(mq, a, smem, grid, st);
+  if (need <= 4) return run<4, PFX>(mq, a, smem, grid, st);
+  if (need <= 8) return run<8, PFX>(mq, a, smem, grid, st);
+  if (need <= 16) return run<16, PFX>(mq, a, smem, grid, st);
+  return run<32, PFX>(mq, a, smem, grid, st);
+}
+
+}  // namespace
+
+cudaError_t launch_gate_tc(const Dims& dm, const void* q, const float* kbar, const float* own,
+                           const int32_t* cu, int32_t* idx, int* status, cudaStream_t st) {
+  return dm.prefix ? launch_impl<true>(dm, q, kbar, own, cu, idx, status, st)
+                   : launch_impl<false>(dm, q, kbar, own, cu, idx, status, st);
 }
 
 }  // namespace moba
