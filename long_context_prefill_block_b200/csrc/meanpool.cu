@@ -53,6 +53,8 @@ __global__ void __launch_bounds__(kThreads) meanpool_kernel(Dims dm, const T* __
   float acc[VEC];
 #pragma unroll
   for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+  // unrolled so that several rows' loads are in flight per thread
+#pragma unroll 8
   for (int j = j0 + rg; j < j1; j += RG) {
     float x[VEC];
     Vec16<T>::load(k + ((start + j) * dm.Hkv + g) * (int64_t)D + lane * VEC, x);
