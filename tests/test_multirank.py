@@ -35,7 +35,7 @@ def _worker(rank, world, port, out):
 
 
 def test_two_ranks_shard_batches_and_take_max_time():
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     port = _free_port()
     mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
