@@ -29,8 +29,10 @@
 //               then per KV tile j O[h] += P_h(j) V(j) and S[h] = Q_h
 //               K(j+1)^T into the same TMEM -- tcgen05.mma operations of one
 //               thread run in issue order, so the PV has read P before the
-//               next QK^T overwrites it. Issuing blocks for about the
-//               group's execution time, hence one issuer per half;
+//               next QK^T overwrites it. The softmax warps hand P over in two
+//               halves (keys 0-63, then 64-127), so the first half's PV runs
+//               while the second half is exponentiated. Issuing blocks for
+//               about the group's execution time, hence one issuer per half;
 //   warp 3      Q loader: cp.async of each half's (gathered, in HIST mode)
 //               query rows into the swizzled layout the MMA reads;
 //   warps 4-7   softmax + epilogue of half 0, warps 8-11 of half 1: one query
@@ -89,7 +91,7 @@ constexpr float kRescaleLog2 = 8.f;
 struct Shared {
   // per query half h
   uint64_t q_full[kQBufs], q_empty[kQBufs];
-  uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+  uint64_t s_full[2], p_lo[2], p_full[2], o_full[2], o_free[2];
   uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
   uint64_t drain[2];
   uint32_t tmem_base;
@@ -290,6 +292,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sh.s_full[i], 1);
+      mbar_init(&sh.p_lo[i], 128);
       mbar_init(&sh.p_full[i], 128);
       mbar_init(&sh.o_full[i], 1);
       mbar_init(&sh.o_free[i], 128);
@@ -404,17 +407,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
               if (j == 0 && uh > 0 &&
                   !(ok = mbar_wait(&sh.o_free[h], (uh - 1) & 1, abort, status)))
                 break;
-              if (!(ok = mbar_wait(&sh.p_full[h], (kh + j) & 1, abort, status))) break;
+              if (!(ok = mbar_wait(&sh.p_lo[h], (kh + j) & 1, abort, status))) break;
             }
             if (!(ok = mbar_wait(&sh.v_full[st], (gg / NS) & 1, abort, status))) break;
             if (j < nh) {
+              // keys 0-63 of P are written first: their PV runs while the
+              // softmax warps still exponentiate keys 64-127
               fence_after_sync();
 #pragma unroll
               for (int kk = 0; kk < TN / 16; ++kk) {
+                if (kk == TN / 32) {
+                  if (!(ok = mbar_wait(&sh.p_full[h], (kh + j) & 1, abort, status))) break;
+                  fence_after_sync();
+                }
                 const uint64_t bd = desc_sw128(sV + st * kTile + kk * 16 * 128, kHalf, 1024);
                 mma_ts(tmem + kOCol + h * 128, tmem + h * 128 + kk * 8, bd, kIdescPV,
                        (j > 0 || kk > 0) ? 1u : 0u);
               }
+              if (!ok) break;
               if (j == nh - 1) commit(&sh.o_full[h]);
             }
             commit(&sh.v_empty[st]);
@@ -625,6 +635,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
             pk[x] = pack_bf16x2(e0, e1);
           }
           tmem_st32(tS + c * 32, pk);
+          if (c == 0) {
+            // keys 0-63 of P are in TMEM: their PV may start
+            tmem_wait_st();
+            fence_before_sync();
+            mbar_arrive(&sh.p_lo[hh]);
+          }
         }
         __syncwarp();
         if (lane == 0) atomicAdd(const_cast<int*>(&exp_cnt[hh]), 1);

@@ -143,10 +143,12 @@ __global__ void __launch_bounds__(kRows) regroup_pass_smem(Dims dm, Chunk ch,
     });
 }
 
-// Exclusive scans of the list sizes and of their tile counts (one CTA).
+// Exclusive scans of the list sizes and of their tile counts (one CTA); the
+// scatter pass's cursors start at zero.
 __global__ void __launch_bounds__(kScanThreads) regroup_scan(int n_lists, int tile_m,
                                                             const int32_t* __restrict__ counts,
-                                                            int32_t* list_off, int32_t* tile_off) {
+                                                            int32_t* list_off, int32_t* tile_off,
+                                                            int32_t* cursor) {
   __shared__ int warp_a[kScanThreads / 32], warp_b[kScanThreads / 32];
   __shared__ int carry_a, carry_b;
   if (threadIdx.x == 0) carry_a = carry_b = 0;
@@ -191,6 +193,7 @@ __global__ void __launch_bounds__(kScanThreads) regroup_scan(int n_lists, int ti
     if (i < n_lists) {
       list_off[i] = pa;
       tile_off[i] = pb;
+      cursor[i] = 0;
     }
     __syncthreads();
     if (threadIdx.x == kScanThreads - 1) {
@@ -221,7 +224,6 @@ cudaError_t launch_regroup(const Dims& dm, const Chunk& ch, const int32_t* idx, 
                            const Regroup& rg, int* status, cudaStream_t st) {
   cudaError_t e;
   if ((e = cudaMemsetAsync(rg.counts, 0, sizeof(int32_t) * ch.n_lists, st))) return e;
-  if ((e = cudaMemsetAsync(rg.cursor, 0, sizeof(int32_t) * ch.n_lists, st))) return e;
   if (dm.batch == 0 || dm.max_seqlen == 0) {
     return cudaMemsetAsync(rg.tile_off + ch.n_lists, 0, sizeof(int32_t), st);
   }
@@ -243,8 +245,9 @@ cudaError_t launch_regroup(const Dims& dm, const Chunk& ch, const int32_t* idx, 
                                                    nullptr, status);
   }
   if ((e = cudaGetLastError())) return e;
+  // the scan also zeroes the scatter pass's cursors
   regroup_scan<<<1, kScanThreads, 0, st>>>(ch.n_lists, ch.tile_m, rg.counts, rg.list_off,
-                                           rg.tile_off);
+                                           rg.tile_off, rg.cursor);
   if ((e = cudaGetLastError())) return e;
   if (smem_lists) {
     regroup_pass_smem<true><<<grid_s, kRows, lsm, st>>>(dm, ch, idx, cu, rg.counts, rg.cursor,
