@@ -632,12 +632,14 @@ def main():
             prev = d_
 
     # ---- dense causal comparison at the same shape
+    # (seconds-long dense passes, as at the million-token shape: one warm-up, one timed)
+    long_dense = ms > 200.0
     dense_out = torch.empty_like(q)
-    for _ in range(2):
+    for _ in range(1 if long_dense else 2):
         moba.dense_causal_forward(q, k, v, cu, max_seqlen=w.max_seqlen, out=dense_out)
     torch.cuda.synchronize(dev)
     d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dreps = 3
+    dreps = 1 if long_dense else 3
     d0.record(stream)
     for _ in range(dreps):
         moba.dense_causal_forward(q, k, v, cu, max_seqlen=w.max_seqlen, out=dense_out)
