@@ -5,8 +5,13 @@ torch provides device memory and the current stream. The binding refuses to
 run if the compiled library is missing; there is no fallback of any kind.
 
 Functions mirror the C ABI of include/moba.h:
-    moba_meanpool, moba_gate_topk, moba_forward, moba_forward_with_indices,
-    dense_causal_forward, moba_workspace_size, moba_device_status.
+    moba_meanpool, moba_meanpool_update, moba_gate_topk, moba_gate_topk_noalloc,
+    moba_forward, moba_forward_with_indices, moba_backward, moba_decode,
+    dense_causal_forward, moba_workspace_size, moba_num_blocks, moba_device_status,
+    moba_selftest_bounded_wait.
+Shapes, element types, devices and (when it is on the host) cu_seqlens are
+checked here before the call: the C ABI takes them on trust, and a mismatch
+would make a kernel read or write past a buffer.
 """
 from __future__ import annotations
 
@@ -113,6 +118,38 @@ def _check_inputs(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError("tensors must be contiguous CUDA tensors")
+    devs = {t.device for t in ts if t is not None}
+    if len(devs) > 1:
+        raise ValueError(f"tensors on different devices: {sorted(map(str, devs))}")
+
+
+def _check_qkv(q, k, v=None, out=None):
+    """Shapes and element types the C ABI takes on trust: a mismatch would make the
+    kernels read or write past the end of a buffer, so it is refused here."""
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("q and k must be [tokens, heads, head_dim]")
+    if k.dtype != q.dtype or (v is not None and v.dtype != q.dtype):
+        raise TypeError(f"q, k, v must share one dtype (got {q.dtype}, {k.dtype}"
+                        f"{'' if v is None else ', ' + str(v.dtype)})")
+    if k.shape[0] != q.shape[0] or k.shape[2] != q.shape[2]:
+        raise ValueError(f"k {tuple(k.shape)} does not match q {tuple(q.shape)}")
+    if q.shape[1] % k.shape[1] != 0:
+        raise ValueError(f"{q.shape[1]} q heads are not a multiple of {k.shape[1]} kv heads")
+    if v is not None and v.shape != k.shape:
+        raise ValueError(f"v {tuple(v.shape)} does not match k {tuple(k.shape)}")
+    if out is not None and (out.shape != q.shape or out.dtype != q.dtype):
+        raise ValueError(f"out must be {tuple(q.shape)} {q.dtype}")
+
+
+def _check_cu(cu_seqlens: torch.Tensor, total_tokens: int) -> None:
+    """cu_seqlens already on the host: starts at 0, never decreases, ends at T."""
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be a 1-D tensor [batch + 1]")
+    if cu_seqlens.is_cuda:
+        return
+    cu = cu_seqlens.to(torch.int64)
+    if int(cu[0]) != 0 or int(cu[-1]) != total_tokens or bool((cu[1:] < cu[:-1]).any()):
+        raise ValueError(f"cu_seqlens must start at 0, not decrease and end at {total_tokens}")
 
 
 def moba_workspace_size(params: MobaParams) -> int:
@@ -130,6 +167,8 @@ def workspace(params: MobaParams, device) -> torch.Tensor:
 def moba_meanpool(k: torch.Tensor, cu_seqlens: torch.Tensor, block_size: int,
                   max_seqlen: Optional[int] = None) -> torch.Tensor:
     """Block means fp32 [batch, num_blocks, Hkv, d]."""
+    _check_qkv(k, k)
+    _check_cu(cu_seqlens, k.shape[0])
     _check_inputs(k)
     p = make_params(k, k, cu_seqlens, block_size, 1, max_seqlen)
     p.num_q_heads = p.num_kv_heads
@@ -146,6 +185,8 @@ def moba_meanpool_update(k_cache: torch.Tensor, cu_seqlens: torch.Tensor, cu_new
                          max_seqlen: Optional[int] = None) -> torch.Tensor:
     """Recompute, in place, the block means kbar [batch, num_blocks, Hkv, d] of the blocks that
     hold each request's last cu_new[r+1] - cu_new[r] cache positions (just appended)."""
+    _check_qkv(k_cache, k_cache)
+    _check_cu(cu_seqlens, k_cache.shape[0])
     _check_inputs(k_cache, kbar)
     p = make_params(k_cache, k_cache, cu_seqlens, block_size, 1, max_seqlen)
     p.num_q_heads = p.num_kv_heads
@@ -176,7 +217,11 @@ def moba_decode(q, k_cache, v_cache, cu_seqlens, cu_q, kbar, block_size: int, to
     """Decode step: request r's queries (rows cu_q[r] .. cu_q[r+1]-1 of q [n, Hq, d]) sit at the
     last positions of its cache (tokens cu_seqlens[r] .. cu_seqlens[r+1]-1 of k_cache, v_cache);
     kbar: the cache's block means. Returns out [n, Hq, d] (and lse [n, Hq], idx [n, Hq, topk])."""
-    _check_inputs(q, k_cache, v_cache, kbar)
+    _check_qkv(k_cache, k_cache, v_cache)
+    if q.dim() != 3 or q.dtype != k_cache.dtype or q.shape[2] != k_cache.shape[2]:
+        raise ValueError("q must be [n, Hq, d] in the cache's dtype and head dim")
+    _check_cu(cu_seqlens, k_cache.shape[0])
+    _check_inputs(q, k_cache, v_cache, kbar, out)
     L = lib()
     p = decode_params(q, k_cache, cu_seqlens, block_size, topk, max_seqlen, shared_routing)
     n = q.shape[0]
@@ -214,6 +259,8 @@ def moba_gate_topk(q, k, cu_seqlens, block_size: int, topk: int, max_seqlen=None
     shared_routing: the q heads of a kv head's group share the blocks of their mean score.
     prefix_mean: the own block is scored by the mean of its keys up to the query and competes
     for the k slots instead of being forced."""
+    _check_qkv(q, k)
+    _check_cu(cu_seqlens, q.shape[0])
     _check_inputs(q, k)
     p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen, shared_routing, prefix_mean)
     cu = _dev_i32(cu_seqlens, q.device)
@@ -231,7 +278,11 @@ def moba_gate_topk_noalloc(q, k, cu_seqlens, block_size: int, topk: int, max_seq
     """moba_gate_topk without a workspace, for callers that cannot allocate
     device memory: the block means use a fixed 4 MiB array inside the
     library (see include/moba.h for the limit and the sharing rules)."""
-    _check_inputs(q, k)
+    _check_qkv(q, k)
+    _check_cu(cu_seqlens, q.shape[0])
+    if idx is not None and (idx.shape != (q.shape[0], q.shape[1], topk) or idx.dtype != torch.int32):
+        raise ValueError(f"idx must be int32 {(q.shape[0], q.shape[1], topk)}")
+    _check_inputs(q, k, idx)
     L = lib()
     fn = L.moba_gate_topk_noalloc
     fn.argtypes = [ctypes.POINTER(MobaParams)] + [ctypes.c_void_p] * 5
@@ -254,7 +305,9 @@ def moba_forward(q, k, v, cu_seqlens, block_size: int, topk: int, max_seqlen=Non
     shared_routing: the q heads of a kv head's group share the blocks of their mean score.
     prefix_mean: the own block is scored by the mean of its keys up to the query and competes
     for the k slots instead of being forced."""
-    _check_inputs(q, k, v)
+    _check_qkv(q, k, v, out)
+    _check_cu(cu_seqlens, q.shape[0])
+    _check_inputs(q, k, v, out)
     p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen, shared_routing, prefix_mean)
     cu = _dev_i32(cu_seqlens, q.device)
     ws = workspace(p, q.device) if ws is None else ws
@@ -272,6 +325,14 @@ def moba_backward(q, k, v, cu_seqlens, out, lse, dout, block_size: int, topk: in
     """Gradients of sum(dout * out) through the chosen blocks: (dq [T,Hq,d], dk, dv [T,Hkv,d])
     in fp32. out, lse: the forward's results; idx: its index rows, or None to run the gate
     again."""
+    _check_qkv(q, k, v, out)
+    _check_cu(cu_seqlens, q.shape[0])
+    if dout.shape != q.shape or dout.dtype != q.dtype:
+        raise ValueError(f"dout must be {tuple(q.shape)} {q.dtype}")
+    if lse.shape != q.shape[:2] or lse.dtype != torch.float32:
+        raise ValueError(f"lse must be float32 {tuple(q.shape[:2])}")
+    if idx is not None and (idx.shape != (q.shape[0], q.shape[1], topk) or idx.dtype != torch.int32):
+        raise ValueError(f"idx must be int32 {(q.shape[0], q.shape[1], topk)}")
     _check_inputs(q, k, v, out, dout, lse, idx)
     L = lib()
     p = make_params(q, k, cu_seqlens, block_size, topk, max_seqlen, shared_routing, prefix_mean)
@@ -298,6 +359,10 @@ def moba_forward_with_indices(q, k, v, cu_seqlens, idx, block_size: int, max_seq
                               prefix_mean: bool = False):
     """MoBA forward with caller-chosen blocks idx int32 [T, Hq, topk] (canonical form; with
     prefix_mean a row may leave out its own block and then reads none of it)."""
+    _check_qkv(q, k, v)
+    _check_cu(cu_seqlens, q.shape[0])
+    if idx.dim() != 3 or idx.shape[:2] != q.shape[:2] or idx.dtype != torch.int32:
+        raise ValueError(f"idx must be int32 [{q.shape[0]}, {q.shape[1]}, topk]")
     _check_inputs(q, k, v, idx)
     p = make_params(q, k, cu_seqlens, block_size, idx.shape[2], max_seqlen, prefix_mean=prefix_mean)
     cu = _dev_i32(cu_seqlens, q.device)
@@ -314,7 +379,9 @@ def moba_forward_with_indices(q, k, v, cu_seqlens, idx, block_size: int, max_seq
 def dense_causal_forward(q, k, v, cu_seqlens, max_seqlen=None, return_lse: bool = False,
                          out: Optional[torch.Tensor] = None):
     """Dense causal attention over each sequence (the comparison kernel)."""
-    _check_inputs(q, k, v)
+    _check_qkv(q, k, v, out)
+    _check_cu(cu_seqlens, q.shape[0])
+    _check_inputs(q, k, v, out)
     p = make_params(q, k, cu_seqlens, 128, 1, max_seqlen)
     cu = _dev_i32(cu_seqlens, q.device)
     out = torch.empty_like(q) if out is None else out
