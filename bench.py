@@ -684,6 +684,9 @@ def main():
     hist_launch_flops = hist_flops / n_pass
     achieved = hist_launch_flops / (hist_launch_ms * 1e-3) / 1e12 if hist_launch_ms > 0 else 0.0
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    # the attention kernels together: history, own block (with its merge), merge
+    attn_ms = stage_ms["attn_history"] + stage_ms["attn_current"] + stage_ms["merge"]
+    attn_tflops = useful / (attn_ms * 1e-3) / 1e12 if attn_ms > 0 else 0.0
     traffic = profile_traffic(os.path.join(ROOT, "long_context_prefill_block_b200", "csrc",
                                            "attn_tc.cu"), w.name)
     tc_path = w.dtype == torch.bfloat16 and w.head_dim == 128 and w.block_size % 128 == 0
@@ -720,6 +723,8 @@ def main():
         "dense_causal_ms": dense_ms,
         "speedup_vs_dense": dense_ms / ms,
         "frac_of_peak_end_to_end": value / world / peak,
+        "attn_kernels_tflops": attn_tflops,
+        "attn_kernels_frac_of_peak": attn_tflops / peak,
     }
     print(json.dumps(line), flush=True)
     if world > 1:
