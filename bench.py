@@ -494,10 +494,13 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     useful, hist_flops, cur_flops, dense_flops = flop_counts(w)
+    elem = 2 if w.dtype == torch.bfloat16 else 4
+    in_bytes = w.total_tokens * (w.num_q_heads + 2 * w.num_kv_heads) * w.head_dim * elem
+    l2_note = ("inputs exceed L2 (q+k+v > 126 MB), no flush" if in_bytes > 126 * 2**20 else
+               f"inputs ({in_bytes / 2**20:.1f} MiB) fit in L2 and stay warm between steps")
     config = {"workload": w.name, "batch": w.batch, "seq_lens": list(w.lengths),
               "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
-              "block_size": w.block_size, "topk": w.topk,
-              "l2": "inputs exceed L2 (q+k+v > 126 MB), no flush"}
+              "block_size": w.block_size, "topk": w.topk, "l2": l2_note}
     if args.variant != "forced":
         config["variant"] = args.variant
     dtype_name = "bf16" if w.dtype == torch.bfloat16 else "f32"
