@@ -205,22 +205,26 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------ CPU oracle leg
-def time_oracle(w, q, k, v, cu, budget_s: float, seed: int = 7):
-    """Time the oracle on a bounded sample of rows; returns (tflops, rows, seconds, threads)."""
+def time_oracle(w, q, k, v, cu, budget_s: float, seed: int = 7, n_rows=None):
+    """Time the oracle on a bounded sample of rows (about budget_s seconds, or
+    n_rows rows when given); returns (tflops, rows, seconds, threads)."""
     import oracle
 
     qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
     total_rows = w.total_tokens * w.num_q_heads
-    n, dt = 64, 0.0
-    while True:  # grow the sample until one call takes a measurable time
-        rows = sample_rows(total_rows, n, seed).numpy()
-        t0 = time.perf_counter()
-        oracle.forward_rows(qc, kc, vc, cu, w.block_size, w.topk, rows)
-        dt = time.perf_counter() - t0
-        if dt > 0.05 * budget_s or n >= total_rows:
-            break
-        n = min(total_rows, n * 8)
-    n2 = int(min(total_rows, max(n, n * budget_s / max(dt, 1e-3))))
+    if n_rows is None:
+        n, dt = 64, 0.0
+        while True:  # grow the sample until one call takes a measurable time
+            rows = sample_rows(total_rows, n, seed).numpy()
+            t0 = time.perf_counter()
+            oracle.forward_rows(qc, kc, vc, cu, w.block_size, w.topk, rows)
+            dt = time.perf_counter() - t0
+            if dt > 0.05 * budget_s or n >= total_rows:
+                break
+            n = min(total_rows, n * 8)
+        n2 = int(min(total_rows, max(n, n * budget_s / max(dt, 1e-3))))
+    else:
+        n2 = int(min(total_rows, n_rows))
     rows = sample_rows(total_rows, n2, seed + 1).numpy()
     t0 = time.perf_counter()
     oracle.forward_rows(qc, kc, vc, cu, w.block_size, w.topk, rows)
@@ -510,9 +514,14 @@ def main():
             return
         q, k, v, cu = make_inputs(w, "cpu")
         per_step = []
-        t_all = time.perf_counter()
-        for _ in range(args.warmup + args.steps):
-            tf, nrows, dt, thr = time_oracle(w, q, k, v, cu, budget_s=2.0)
+        # about two minutes of oracle work for the whole run, at most 2 s a step;
+        # the first step sizes the row sample, the others reuse its size
+        n_steps = args.warmup + args.steps
+        budget = min(2.0, max(0.05, 120.0 / max(1, n_steps)))
+        n_rows = None
+        for _ in range(n_steps):
+            tf, nrows, dt, thr = time_oracle(w, q, k, v, cu, budget_s=budget, n_rows=n_rows)
+            n_rows = nrows
             per_step.append((tf, nrows, dt))
         per_step = per_step[args.warmup:]
         tf = float(np.mean([x[0] for x in per_step]))
