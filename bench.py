@@ -73,6 +73,16 @@ def flop_counts(w):
     return useful, hist, cur, dense
 
 
+def gate_flops(w):
+    """Gate scoring FLOPs of one layer-forward, reported apart from the useful
+    attention FLOPs: 2*d per (query, head, complete earlier block scored)."""
+    total = 0
+    for n in w.lengths:
+        c = np.arange(n, dtype=np.int64) // w.block_size
+        total += int(c.sum()) * 2 * w.head_dim * w.num_q_heads
+    return total
+
+
 def flops_from_indices(idx, cu, B, d):
     """(history, own-block) useful FLOPs of index rows idx [T, Hq, k] (device
     tensor): every chosen earlier block gives B keys, the own block, when
@@ -732,6 +742,7 @@ def main():
         "clocks": clock_info,
         "stage_ms": stage_ms,
         "useful_flop_per_step": useful,
+        "gate_flop_per_step": gate_flops(w),
         "dense_causal_ms": dense_ms,
         "speedup_vs_dense": dense_ms / ms,
         "frac_of_peak_end_to_end": value / world / peak,

@@ -68,3 +68,11 @@ def test_flops_equal_the_keys_the_oracle_selects(lengths, B, topk):
     assert (fh, fc) == (hist, cur)
     rows = np.arange(sum(lengths) * Hq)
     assert bench.row_flops(w, rows) == useful
+
+
+def test_gate_flops_count_the_complete_earlier_blocks():
+    # 2 * d per scored block: query p of block c scores blocks 0 .. c-1
+    w = Workload("g", (1000, 1), 3, 1, 64, 128, 3, torch.float32, 0, 1.0, 0.3)
+    scored = sum(p // 128 for p in range(1000))
+    assert bench.gate_flops(w) == 2 * 64 * 3 * scored
+    assert bench.gate_flops(WORKLOADS["llama_1m"]) == 2 * 128 * 32 * 4096 * (256 * 255 // 2)
