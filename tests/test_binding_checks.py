@@ -78,3 +78,19 @@ def test_consistent_cpu_arguments_reach_the_device_check():
     q, k, v = _qkv()
     with pytest.raises(ValueError, match="CUDA"):
         moba.moba_forward(q, k, v, CU, 32, 2)
+
+
+def test_decode_and_meanpool_arguments_are_checked():
+    _, k, v = _qkv()
+    q = torch.zeros(2, HQ, D, dtype=torch.bfloat16)
+    kbar = torch.zeros(2, 2, HKV, D)
+    cu_q = torch.tensor([0, 1, 2], dtype=torch.int32)
+    with pytest.raises(ValueError):   # q head dim differs from the cache's
+        moba.moba_decode(torch.zeros(2, HQ, 64, dtype=torch.bfloat16), k, v, CU, cu_q, kbar, 32, 2)
+    with pytest.raises(TypeError):    # cache K and V of different dtypes
+        moba.moba_decode(q, k, v.float(), CU, cu_q, kbar, 32, 2)
+    with pytest.raises(ValueError, match="cu_seqlens"):
+        moba.moba_meanpool(k, torch.tensor([0, 10], dtype=torch.int32), 32)
+    with pytest.raises(ValueError, match="cu_seqlens"):
+        moba.moba_meanpool_update(k, torch.tensor([0, 70], dtype=torch.int32),
+                                  torch.tensor([0, 1], dtype=torch.int32), kbar, 32, 1)
