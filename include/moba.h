@@ -127,13 +127,15 @@ MOBA_API moba_status moba_gate_topk(const moba_params* p, const void* q, const v
  * the library, which every GPU that loads the library holds until the
  * process exits. It calls no allocating routine.
  * Limit: batch * moba_num_blocks(p) * Hkv * d * 4 bytes must not exceed
- * 4 MiB, else MOBA_ERR_WORKSPACE is returned and nothing is launched.
+ * 4 MiB, else MOBA_ERR_WORKSPACE is returned and nothing is launched; this
+ * check comes before the pointer checks, so it does not depend on them.
  * The first call on a device looks up the array's device address (with that
  * device current); make that first call before any stream capture.
  * All calls share the one array and it keeps the last call's contents
  * (nothing in it has to start at zero); calls that overlap on the GPU --
  * on different streams, or from different host threads -- race on it.
- * Device-side checks of cu_seqlens are not recorded in the status word.
+ * A sequence longer than max_seqlen is skipped and recorded in the status
+ * word (moba_device_status), as moba_gate_topk does.
  * own_block = 1 needs workspace for its scores: MOBA_ERR_UNSUPPORTED. */
 MOBA_API moba_status moba_gate_topk_noalloc(const moba_params* p, const void* q, const void* k,
                                             const int32_t* cu_seqlens, int32_t* idx,

@@ -5,8 +5,7 @@
 #include <cstdint>
 #include <cstring>
 
-#include "common.cuh"
-#include "moba.h"
+#include "host_api.cuh"
 
 namespace moba {
 // Per-device status word; kernels get its address, never the symbol.
@@ -25,17 +24,6 @@ cudaError_t launch_dense_tc(const Dims& dm, const void* q, const void* k, const 
 bool tc_supported(const Dims& dm);
 cudaError_t launch_wait_selftest(int* status, int* done, cudaStream_t st);
 int tc_tile_m();
-}  // namespace moba
-
-using namespace moba;
-
-namespace {
-
-// Partial results are kept for at most this many bytes per pass; larger
-// problems are processed one group of kv heads at a time.
-constexpr size_t kPartialCap = size_t(32) << 30;
-
-size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 moba_status validate(const moba_params* p, Dims& dm) {
   if (!p) return MOBA_ERR_INVALID_ARG;
@@ -65,6 +53,24 @@ moba_status validate(const moba_params* p, Dims& dm) {
   dm.prefix = p->own_block;
   return MOBA_OK;
 }
+
+int* status_word() {
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) return nullptr;
+  return static_cast<int*>(ptr);
+}
+
+}  // namespace moba
+
+using namespace moba;
+
+namespace {
+
+// Partial results are kept for at most this many bytes per pass; larger
+// problems are processed one group of kv heads at a time.
+constexpr size_t kPartialCap = size_t(32) << 30;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; }
 
@@ -130,12 +136,6 @@ Layout plan(const Dims& dm, bool own_idx) {
   L.part_lse = take(sizeof(float) * prows);
   L.total = off;
   return L;
-}
-
-int* status_word() {
-  void* ptr = nullptr;
-  if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) return nullptr;
-  return static_cast<int*>(ptr);
 }
 
 moba_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA; }

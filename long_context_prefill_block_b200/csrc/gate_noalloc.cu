@@ -14,11 +14,12 @@
 // the library holds it until the process exits. In host code its name is
 // only a host-side stand-in, not a device address, so the device address is
 // looked up with cudaGetSymbolAddress once per device, with that device
-// current, and cached.
+// current, and cached. The status word (a __device__ symbol of api.cu) is
+// reached the same way, so bad sequence offsets are reported as they are
+// for moba_gate_topk; nothing here allocates.
 #include <mutex>
 
-#include "common.cuh"
-#include "moba.h"
+#include "host_api.cuh"
 
 namespace {
 
@@ -32,10 +33,11 @@ static __device__ __align__(256) float g_gate_scratch[kScratchBytes / sizeof(flo
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 float* g_scratch_ptr[kMaxDevices] = {};
+int* g_status_ptr[kMaxDevices] = {};
 
-// Device address of g_gate_scratch on the current device; the first call on
-// a device performs the lookup.
-cudaError_t scratch_on_current_device(float** out) {
+// Device addresses of g_gate_scratch and of the status word on the current
+// device; the first call on a device performs the lookups.
+cudaError_t addresses_on_current_device(float** scratch, int** status) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -45,40 +47,14 @@ cudaError_t scratch_on_current_device(float** out) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_gate_scratch);
     if (e != cudaSuccess) return e;
+    int* st = moba::status_word();
+    if (!st) return cudaErrorInvalidSymbol;
+    g_status_ptr[dev] = st;
     g_scratch_ptr[dev] = static_cast<float*>(ptr);
   }
-  *out = g_scratch_ptr[dev];
+  *scratch = g_scratch_ptr[dev];
+  *status = g_status_ptr[dev];
   return cudaSuccess;
-}
-
-moba_status dims_of(const moba_params* p, moba::Dims& dm) {
-  if (!p) return MOBA_ERR_INVALID_ARG;
-  if (p->batch < 0 || p->total_tokens < 0 || p->max_seqlen < 0 || p->num_q_heads <= 0 ||
-      p->num_kv_heads <= 0 || p->num_q_heads % p->num_kv_heads != 0 || p->block_size <= 0 ||
-      p->topk <= 0)
-    return MOBA_ERR_INVALID_ARG;
-  if (p->routing != 0 && p->routing != 1) return MOBA_ERR_INVALID_ARG;
-  if (p->own_block != 0 && p->own_block != 1) return MOBA_ERR_INVALID_ARG;
-  // the prefix-mean gate keeps T * Hq own-block scores: no room in the fixed array
-  if (p->own_block) return MOBA_ERR_UNSUPPORTED;
-  if (p->dtype != MOBA_BF16 && p->dtype != MOBA_F32) return MOBA_ERR_UNSUPPORTED;
-  if (p->head_dim != 64 && p->head_dim != 128) return MOBA_ERR_UNSUPPORTED;
-  if (p->topk > 32) return MOBA_ERR_UNSUPPORTED;
-  if ((int64_t)p->total_tokens * p->num_q_heads * p->topk >= (int64_t(1) << 31))
-    return MOBA_ERR_UNSUPPORTED;
-  dm.batch = p->batch;
-  dm.T = p->total_tokens;
-  dm.max_seqlen = p->max_seqlen;
-  dm.Hq = p->num_q_heads;
-  dm.Hkv = p->num_kv_heads;
-  dm.d = p->head_dim;
-  dm.B = p->block_size;
-  dm.topk = p->topk;
-  dm.nb = (int)(((int64_t)p->max_seqlen + p->block_size - 1) / p->block_size);
-  dm.dtype = p->dtype == MOBA_BF16 ? moba::kBF16 : moba::kF32;
-  dm.shared = p->routing;
-  dm.prefix = 0;
-  return MOBA_OK;
 }
 
 bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; }
@@ -89,21 +65,26 @@ extern "C" moba_status moba_gate_topk_noalloc(const moba_params* p, const void* 
                                               const int32_t* cu_seqlens, int32_t* idx,
                                               void* stream) {
   moba::Dims dm;
-  const moba_status s = dims_of(p, dm);
+  const moba_status s = moba::validate(p, dm);
   if (s != MOBA_OK) return s;
+  // the prefix-mean gate keeps T * Hq own-block scores: no room in the fixed array
+  if (dm.prefix) return MOBA_ERR_UNSUPPORTED;
   if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
-  if (!q || !k || !cu_seqlens || !idx || !aligned16(q) || !aligned16(k))
-    return MOBA_ERR_INVALID_ARG;
+  // the size limit is checked before the pointers, so that a refusal never
+  // depends on what the pointers hold
   const size_t need = sizeof(float) * (size_t)dm.batch * dm.nb * dm.Hkv * dm.d;
   if (need > kScratchBytes) return MOBA_ERR_WORKSPACE;  // beyond the built-in 4 MiB
+  if (!q || !k || !cu_seqlens || !idx || !aligned16(q) || !aligned16(k))
+    return MOBA_ERR_INVALID_ARG;
   float* kbar = nullptr;
-  if (scratch_on_current_device(&kbar) != cudaSuccess) return MOBA_ERR_CUDA;
+  int* status = nullptr;
+  if (addresses_on_current_device(&kbar, &status) != cudaSuccess) return MOBA_ERR_CUDA;
   // Nothing has to start at zero: the mean-pool writes every slot of the
   // table that the gate reads (0 for blocks past a sequence's end).
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (moba::launch_meanpool(dm, k, cu_seqlens, kbar, nullptr, st) != cudaSuccess)
+  if (moba::launch_meanpool(dm, k, cu_seqlens, kbar, status, st) != cudaSuccess)
     return MOBA_ERR_CUDA;
-  if (moba::launch_gate(dm, q, kbar, nullptr, cu_seqlens, idx, nullptr, st) != cudaSuccess)
+  if (moba::launch_gate(dm, q, kbar, nullptr, cu_seqlens, idx, status, st) != cudaSuccess)
     return MOBA_ERR_CUDA;
   return MOBA_OK;
 }
