@@ -7,8 +7,9 @@
 
 A step runs the whole path -- block mean-pool, gate/top-k, regrouping,
 history and own-block attention, merge -- on seeded synthetic inputs of the
-named workload (default: the scaling-law shape, batch 4 x 8192 tokens, 16
-heads, d=128, B=512, k=3, bf16). Inputs stay resident in HBM; they are larger
+named workload (default: the Llama-3.1-8B million-token prefill shape, 1 x
+1,048,576 tokens, 32 q / 8 kv heads, d=128, B=4096, k=12, bf16: the largest
+workload that fits one GPU). Inputs stay resident in HBM; they are larger
 than the 126 MB L2, so no flush is needed between steps.
 
 Metric: useful TFLOP/s (only QK^T and PV over the selected keys, 4*d per
@@ -17,8 +18,14 @@ rank runs the same workload on its own GPU (weak scaling, no collective on
 the data path); `value` is the sum of all ranks' useful FLOPs divided by the
 slowest rank's time. Prints one JSON line on rank 0.
 
+The roofline fraction divides by the measured bf16 peak: the sustained
+figure when the timed region lasts a second or more (the kernel then runs
+under the power cap), else the burst figure; both fractions are reported.
+
 --impl reference times the fp64 CPU oracle (the only reference this method
-has) on a bounded sample of the same workload on the host cores.
+has) on a bounded sample of the same workload on the host cores, with the
+same input bits as the GPU arm (drawn on the GPU when one is present; only
+K, V and the sampled q rows are copied to the host).
 
 --variant picks the gate: forced own block (default, the headline), shared
 (one choice per kv head's group, by the group's mean score) or prefix (the
@@ -34,6 +41,7 @@ keys' K and V, the scored block means, q and out) against the HBM peak.
 from __future__ import annotations
 
 import argparse
+import concurrent.futures as cf
 import ctypes
 import hashlib
 import json
@@ -54,7 +62,9 @@ sys.path.insert(0, ROOT)
 from moba_inputs import WORKLOADS, make_inputs, sample_rows  # noqa: E402
 
 METRIC = "moba_prefill_fwd_useful_tflops"
-FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+DEFAULT_WORKLOAD = "llama_1m"
+TIE_GAP = 1e-4  # near-tie band of the block indices (relative score gap)
 
 
 # ------------------------------------------------------------ accounting
@@ -81,6 +91,29 @@ def gate_flops(w):
         c = np.arange(n, dtype=np.int64) // w.block_size
         total += int(c.sum()) * 2 * w.head_dim * w.num_q_heads
     return total
+
+
+def history_pairs(w):
+    """(query, head, chosen earlier block) entries of one forward with the forced own block."""
+    total = 0
+    for n in w.lengths:
+        c = np.arange(n, dtype=np.int64) // w.block_size
+        total += int(np.minimum(w.topk - 1, c).sum()) * w.num_q_heads
+    return total
+
+
+def stage_bytes(w):
+    """Algorithmic HBM bytes of the memory-bound stages of one forward:
+    mean-pool reads K once and writes the block means; the gate reads Q once
+    and writes the index rows; regroup reads the index rows twice (count and
+    scatter passes) and writes one 4-byte entry per history pair."""
+    esz = 2 if w.dtype == torch.bfloat16 else 4
+    T, Hq, Hkv, d, k = w.total_tokens, w.num_q_heads, w.num_kv_heads, w.head_dim, w.topk
+    nb = sum((n + w.block_size - 1) // w.block_size for n in w.lengths)
+    idx_bytes = T * Hq * k * 4
+    return {"meanpool": T * Hkv * d * esz + nb * Hkv * d * 4,
+            "gate_topk": T * Hq * d * esz + idx_bytes,
+            "regroup": 2 * idx_bytes + 4 * history_pairs(w)}
 
 
 def flops_from_indices(idx, cu, B, d):
@@ -136,6 +169,15 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def tensor_peak(peaks, timed_s: float):
+    """(peak TFLOP/s, which one): the sustained bf16 figure for a timed region
+    of a second or more (the GPU then runs under its power cap), else the
+    burst figure."""
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sustained = float(peaks.get("bf16_tflops_sustained", burst))
+    return (sustained, "sustained") if timed_s >= 1.0 else (burst, "burst")
+
+
 def profile_traffic(kernel_src: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the current source of the kernel; else None."""
@@ -149,6 +191,27 @@ def profile_traffic(kernel_src: str, workload: str):
         return None
     sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
     return float(m.group(1)) if sha.startswith(s.group(1)) else None
+
+
+def sha256_of(t: torch.Tensor) -> str:
+    """SHA-256 of a host tensor's stored bytes."""
+    x = t.detach().contiguous()
+    if x.dtype == torch.bfloat16:
+        x = x.view(torch.int16)
+    return hashlib.sha256(memoryview(x.numpy()).cast("B")).hexdigest()
+
+
+def input_hashes(named):
+    """{name: sha256} of host tensors, hashed in parallel (hashlib releases the GIL)."""
+    with cf.ThreadPoolExecutor(max_workers=len(named)) as ex:
+        futs = {n: ex.submit(sha256_of, t) for n, t in named.items()}
+        return {n: f.result() for n, f in futs.items()}
+
+
+def pinned_copy(x: torch.Tensor) -> torch.Tensor:
+    h = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    h.copy_(x)
+    return h
 
 
 # ------------------------------------------------------------ clocks
@@ -215,20 +278,37 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------ CPU oracle leg
-def time_oracle(w, q, k, v, cu, budget_s: float, seed: int = 7, n_rows=None):
+def q_rows_from(q: torch.Tensor):
+    """Function rows -> the host copy of those q rows (row = t * Hq + h) of q,
+    which may live on the GPU: only the sampled rows cross to the host."""
+    flat = q.reshape(-1, q.shape[-1])
+
+    def take(rows):
+        sel = torch.as_tensor(np.asarray(rows, dtype=np.int64), device=q.device)
+        return flat[sel].cpu()
+
+    return take
+
+
+def time_oracle(w, kc, vc, cu, q_rows_of, budget_s: float, seed: int = 7, n_rows=None):
     """Time the oracle on a bounded sample of rows (about budget_s seconds, or
-    n_rows rows when given); returns (tflops, rows, seconds, threads)."""
+    n_rows rows when given). kc, vc: host K and V; q_rows_of(rows): host q rows.
+    Returns dict(tflops, rows, seconds, threads, result=(out, lse, idx, gap), q_rows)."""
     import oracle
 
-    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
     total_rows = w.total_tokens * w.num_q_heads
+
+    def run(rows):
+        qr = q_rows_of(rows)
+        t0 = time.perf_counter()
+        res = oracle.forward_rows(None, kc, vc, cu, w.block_size, w.topk, rows, q_rows=qr,
+                                  num_q_heads=w.num_q_heads)
+        return res, qr, time.perf_counter() - t0
+
     if n_rows is None:
-        n, dt = 64, 0.0
+        n = 64
         while True:  # grow the sample until one call takes a measurable time
-            rows = sample_rows(total_rows, n, seed).numpy()
-            t0 = time.perf_counter()
-            oracle.forward_rows(qc, kc, vc, cu, w.block_size, w.topk, rows)
-            dt = time.perf_counter() - t0
+            _, _, dt = run(sample_rows(total_rows, n, seed).numpy())
             if dt > 0.05 * budget_s or n >= total_rows:
                 break
             n = min(total_rows, n * 8)
@@ -236,10 +316,61 @@ def time_oracle(w, q, k, v, cu, budget_s: float, seed: int = 7, n_rows=None):
     else:
         n2 = int(min(total_rows, n_rows))
     rows = sample_rows(total_rows, n2, seed + 1).numpy()
-    t0 = time.perf_counter()
-    oracle.forward_rows(qc, kc, vc, cu, w.block_size, w.topk, rows)
-    dt = time.perf_counter() - t0
-    return row_flops(w, rows) / dt / 1e12, len(rows), dt, oracle.num_threads()
+    res, qr, dt = run(rows)
+    return {"tflops": row_flops(w, rows) / dt / 1e12, "rows": rows, "seconds": dt,
+            "threads": oracle.num_threads(), "result": res, "q_rows": qr}
+
+
+def parity_stats(w, leg, kc, vc, cu, got_out, got_lse, got_idx):
+    """The GPU forward against the oracle on the CPU leg's sampled rows:
+    output and lse errors, index mismatches (and how many fall outside the
+    near-tie band), near-tie count and a histogram of the top-k margins (the
+    oracle's relative score gap between the last chosen and the first rejected
+    earlier block; "none" where no earlier block was rejected)."""
+    import oracle
+
+    ref, ref_lse, ref_idx, gap = (np.array(x) for x in leg["result"])
+    rows = leg["rows"]
+    mism = np.nonzero((got_idx != ref_idx).any(axis=1))[0]
+    beyond = int((gap[mism] >= TIE_GAP).sum())
+    if len(mism):
+        # near-tie rows: the oracle with the GPU's own choice
+        o2, l2, _, _ = oracle.forward_rows(None, kc, vc, cu, w.block_size, w.topk, rows[mism],
+                                           indices=got_idx[mism], q_rows=leg["q_rows"][mism],
+                                           num_q_heads=w.num_q_heads)
+        ref[mism] = o2
+        ref_lse[mism] = l2
+    err = np.abs(got_out.astype(np.float64) - ref)
+    lerr = np.abs(got_lse.astype(np.float64) - ref_lse)
+    finite = gap[np.isfinite(gap)]
+    edges = [0.0, 1e-6, 1e-5, 1e-4, 1e-3, 1e-2, 1e-1, np.inf]
+    names = ["<1e-6", "1e-6..1e-5", "1e-5..1e-4", "1e-4..1e-3", "1e-3..1e-2", "1e-2..1e-1",
+             ">=1e-1"]
+    counts, _ = np.histogram(finite, bins=edges)
+    hist = {n: int(c) for n, c in zip(names, counts)}
+    hist["none"] = int((~np.isfinite(gap)).sum())
+    tol = (2e-2, 2e-3) if w.dtype == torch.bfloat16 else (1e-4, 1e-4)
+    return {"rows": int(len(rows)), "max_abs_err": float(err.max()),
+            "mean_abs_err": float(err.mean()), "lse_max_abs_err": float(lerr.max()),
+            "index_mismatch_rows": int(len(mism)), "index_mismatch_beyond_tie": beyond,
+            "near_tie_rows": int((gap < TIE_GAP).sum()), "topk_margin_hist": hist,
+            "tolerance": {"max_abs": tol[0], "mean_abs": tol[1], "tie_gap": TIE_GAP},
+            "pass": bool(beyond == 0 and err.max() <= tol[0] and err.mean() <= tol[1])}
+
+
+def reference_inputs(w):
+    """Inputs of the reference arm with the GPU arm's bits: drawn on the GPU
+    when one is present (then only K, V and sampled q rows go to the host),
+    else on the host."""
+    if torch.cuda.is_available():
+        dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+        torch.cuda.set_device(dev)
+        q, k, v, cu = make_inputs(w, dev)
+        kc, vc = k.cpu(), v.cpu()
+        del k, v
+        return q, kc, vc, cu, "drawn on the GPU (the GPU arm's bits)"
+    q, k, v, cu = make_inputs(w, "cpu")
+    return q, k, v, cu, "drawn on the host (no GPU present)"
 
 
 # ------------------------------------------------------------ main
@@ -308,9 +439,9 @@ def bench_backward(args, w, moba, q, k, v, cu, dev, world, rank, config, shared,
     ms = reduce_max(e0.elapsed_time(e1) / args.steps, world, dev)
 
     # end to end: the step's inputs from pinned host memory, the gradients back
-    host_in = [x.cpu().pin_memory() for x in (q, k, v, out, lse, dout, idx)]
+    host_in = [pinned_copy(x) for x in (q, k, v, out, lse, dout, idx)]
     dev_in = [torch.empty_like(x) for x in (q, k, v, out, lse, dout, idx)]
-    host_out = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in (dq, dk, dv)]
+    host_out = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (dq, dk, dv)]
 
     def e2e_step():
         for d_, h_ in zip(dev_in, host_in):
@@ -322,7 +453,7 @@ def bench_backward(args, w, moba, q, k, v, cu, dev, world, rank, config, shared,
     for _ in range(2):
         e2e_step()
     torch.cuda.synchronize(dev)
-    erep = max(3, min(args.steps, 10))
+    erep = 3 if ms > 100 else max(3, min(args.steps, 10))
     e0.record(stream)
     for _ in range(erep):
         e2e_step()
@@ -334,7 +465,7 @@ def bench_backward(args, w, moba, q, k, v, cu, dev, world, rank, config, shared,
             torch.distributed.destroy_process_group()
         return
     peaks, peak_src = load_peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak, which = tensor_peak(peaks, ms * args.steps * 1e-3)
     value = useful * world / (ms * 1e-3) / 1e12
     line = {
         "metric": "moba_prefill_bwd_useful_tflops", "value": value, "unit": "TFLOP/s",
@@ -345,7 +476,7 @@ def bench_backward(args, w, moba, q, k, v, cu, dev, world, rank, config, shared,
         "roofline": {"bound": "tensor", "achieved": value / world, "peak": peak,
                      "unit": "TFLOP/s", "frac": value / world / peak, "traffic": None,
                      "kernel": "moba_backward, all launches (a lower bound for each kernel)",
-                     "peak_source": f"{peak_src} bf16 burst"},
+                     "peak_source": f"{peak_src} bf16 {which}"},
         "cpu_baseline": None,
         "e2e": {"value": useful * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms,
@@ -440,8 +571,8 @@ def bench_decode(args, w, moba, q_all, k, v, cu, dev, world, rank, config, share
     clock_info = clocks.summarise(t_lo, t_hi) if clocks else None
     ms = reduce_max(e0.elapsed_time(e1) / args.steps, world, dev)
     # end to end: the step's query rows in from pinned memory, the outputs back
-    hq = q.cpu().pin_memory()
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hq = pinned_copy(q)
+    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     dq = torch.empty_like(q)
 
     def e2e_step():
@@ -489,15 +620,50 @@ def bench_decode(args, w, moba, q_all, k, v, cu, dev, world, rank, config, share
         torch.distributed.destroy_process_group()
 
 
+def run_reference(args, w, config):
+    """--impl reference: the fp64 oracle on the host cores, each step a
+    bounded seeded row sample of the workload, same input bits as the GPU arm."""
+    q, kc, vc, cu, origin = reference_inputs(w)
+    take = q_rows_from(q)
+    per_step = []
+    # about two minutes of oracle work for the whole run, at most 2 s a step;
+    # the first step sizes the row sample, the others reuse its size
+    n_steps = args.warmup + args.steps
+    budget = min(2.0, max(0.05, 120.0 / max(1, n_steps)))
+    n_rows = None
+    thr = 0
+    for i in range(n_steps):
+        leg = time_oracle(w, kc, vc, cu, take, budget_s=budget, n_rows=n_rows, seed=7 + i)
+        n_rows = len(leg["rows"])
+        thr = leg["threads"]
+        per_step.append((leg["tflops"], n_rows, leg["seconds"]))
+    per_step = per_step[args.warmup:]
+    tf = float(np.mean([x[0] for x in per_step]))
+    ms = float(np.mean([x[2] for x in per_step])) * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": tf, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+            "cpu_baseline": {"kind": "oracle", "value": tf, "unit": "TFLOP/s", "cores": thr,
+                             "sample": f"{per_step[0][1]} seeded (token, head) rows per step "
+                                       f"of {w.name} (inputs {origin}), useful FLOPs of those "
+                                       "rows"},
+            "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: about 10 s of work, 3..400 steps)")
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="scaling_8k", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-hash", action="store_true", help="skip the input SHA-256s")
     ap.add_argument("--variant", default="forced", choices=["forced", "shared", "prefix"])
     ap.add_argument("--pass", dest="pass_", default="forward",
                     choices=["forward", "backward", "decode"])
@@ -522,31 +688,9 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        q, k, v, cu = make_inputs(w, "cpu")
-        per_step = []
-        # about two minutes of oracle work for the whole run, at most 2 s a step;
-        # the first step sizes the row sample, the others reuse its size
-        n_steps = args.warmup + args.steps
-        budget = min(2.0, max(0.05, 120.0 / max(1, n_steps)))
-        n_rows = None
-        for _ in range(n_steps):
-            tf, nrows, dt, thr = time_oracle(w, q, k, v, cu, budget_s=budget, n_rows=n_rows)
-            n_rows = nrows
-            per_step.append((tf, nrows, dt))
-        per_step = per_step[args.warmup:]
-        tf = float(np.mean([x[0] for x in per_step]))
-        ms = float(np.mean([x[2] for x in per_step])) * 1e3
-        line = {"impl": "reference", "metric": METRIC, "value": tf, "unit": "TFLOP/s",
-                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
-                "cpu_baseline": {"kind": "oracle", "value": tf, "unit": "TFLOP/s", "cores": thr,
-                                 "sample": f"{per_step[0][1]} seeded (token, head) rows per step "
-                                           f"of {w.name}, useful FLOPs of those rows"},
-                "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
-        return
+        if args.steps is None:
+            args.steps = 10
+        return run_reference(args, w, config)
 
     import long_context_prefill_block_b200 as moba
 
@@ -562,10 +706,12 @@ def main():
     cu_d = cu.to(dev)
     shared, prefix = args.variant == "shared", args.variant == "prefix"
     if args.pass_ == "backward":
+        args.steps = args.steps or 20
         return bench_backward(args, w, moba, q, k, v, cu, dev, world, rank, config, shared, prefix)
     if args.pass_ == "decode":
         if prefix:
             raise ValueError("the decode step takes the forced own block only")
+        args.steps = args.steps or 200
         return bench_decode(args, w, moba, q, k, v, cu, dev, world, rank, config, shared)
     p = moba.make_params(q, k, cu, w.block_size, w.topk, w.max_seqlen, shared, prefix)
     ws = moba.workspace(p, dev)
@@ -580,14 +726,16 @@ def main():
     L = moba.lib()
     P = ctypes.byref(p)
     sp = ctypes.c_void_p(stream.cuda_stream)
+    vp = lambda x: ctypes.c_void_p(x.data_ptr())
 
-    def step():
-        rc = L.moba_forward(P, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
-                            ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(cu_d.data_ptr()),
-                            ctypes.c_void_p(out.data_ptr()), None, ctypes.c_void_p(ws.data_ptr()),
-                            ws.numel(), sp)
+    def forward(qq, kk, vv, oo, s=sp):
+        rc = L.moba_forward(P, vp(qq), vp(kk), vp(vv), vp(cu_d), vp(oo), None, vp(ws),
+                            ws.numel(), s)
         if rc:
             raise RuntimeError(f"moba_forward failed: {rc}")
+
+    def step():
+        forward(q, k, v, out)
 
     def barrier():
         if world > 1:
@@ -599,11 +747,16 @@ def main():
     clocks = ClockSampler(dev.index) if rank == 0 else None
     if clocks:
         clocks.wait_first_sample()
+    t_w = time.perf_counter()
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize(dev)
+    warm_s = (time.perf_counter() - t_w) / max(args.warmup, 3)
     if moba.moba_device_status(dev) != 0:
         raise RuntimeError("device status error after warm-up")
+    if args.steps is None:  # about ten seconds of timed work, 3 to 400 steps
+        args.steps = int(min(400, max(3, round(10.0 / max(warm_s, 1e-4)))))
+        args.steps = int(max_over_ranks(args.steps))
 
     # ---- timed region: K steps, barrier + sync on both sides
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -622,6 +775,7 @@ def main():
     clock_info = clocks.summarise(t_lo, t_hi) if clocks else None
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
     value = useful * world / (ms * 1e-3) / 1e12
+    long_step = ms > 100.0
 
     # ---- per-stage timing (same stream, CUDA events recorded by the library)
     n_pass = L.moba_num_passes(P)
@@ -633,12 +787,10 @@ def main():
     ev_arr = (ctypes.c_void_p * n_ev)(*[ctypes.c_void_p(e.cuda_event) for e in evs])
     stage_ms = {"meanpool": 0.0, "gate_topk": 0.0, "regroup": 0.0, "attn_history": 0.0,
                 "attn_current": 0.0, "merge": 0.0}
-    reps = max(3, min(args.steps, 10))
+    reps = 3 if long_step else max(3, min(args.steps, 10))
     for _ in range(reps):
-        rc = L.moba_forward_staged(P, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
-                                   ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(cu_d.data_ptr()),
-                                   ctypes.c_void_p(out.data_ptr()), None,
-                                   ctypes.c_void_p(ws.data_ptr()), ws.numel(), ev_arr, n_ev, sp)
+        rc = L.moba_forward_staged(P, vp(q), vp(k), vp(v), vp(cu_d), vp(out), None, vp(ws),
+                                   ws.numel(), ev_arr, n_ev, sp)
         if rc:
             raise RuntimeError(f"moba_forward_staged failed: {rc}")
         torch.cuda.synchronize(dev)
@@ -670,47 +822,76 @@ def main():
     dense_ms = d0.elapsed_time(d1) / dreps
     del dense_out
 
-    # ---- end to end through the public API with host buffers
-    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
-    hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    # ---- end to end through the C ABI with host buffers: every step copies
+    # its q, k, v in from pinned host memory and its output back. Two device
+    # buffer sets let step i+1's input copies and step i-1's output copy run
+    # on their own streams while step i computes.
+    hq, hk, hv = (pinned_copy(x) for x in (q, k, v))
+    hout = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    bufs = [(q, k, v, out), tuple(torch.empty_like(x) for x in (q, k, v, out))]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_fwd = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    started = [False, False]
 
-    def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        rc = L.moba_forward(P, ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()),
-                            ctypes.c_void_p(dv.data_ptr()), ctypes.c_void_p(cu_d.data_ptr()),
-                            ctypes.c_void_p(out.data_ptr()), None, ctypes.c_void_p(ws.data_ptr()),
-                            ws.numel(), sp)
-        if rc:
-            raise RuntimeError(f"moba_forward failed: {rc}")
-        hout.copy_(out, non_blocking=True)
+    def e2e_steps(n):
+        for i in range(n):
+            s = i % 2
+            bq, bk, bv, bo = bufs[s]
+            if i == 0:
+                s_in.wait_stream(stream)  # the copies start after the timing event
+            if started[s]:
+                s_in.wait_event(ev_fwd[s])  # the forward that last read this buffer set
+            with torch.cuda.stream(s_in):
+                bq.copy_(hq, non_blocking=True)
+                bk.copy_(hk, non_blocking=True)
+                bv.copy_(hv, non_blocking=True)
+                ev_in[s].record(s_in)
+            stream.wait_event(ev_in[s])
+            if started[s]:
+                stream.wait_event(ev_out[s])  # the output copy that last read this buffer
+            forward(bq, bk, bv, bo)
+            ev_fwd[s].record(stream)
+            s_out.wait_event(ev_fwd[s])
+            with torch.cuda.stream(s_out):
+                hout.copy_(bo, non_blocking=True)
+                ev_out[s].record(s_out)
+            started[s] = True
+        stream.wait_stream(s_out)
 
-    for _ in range(2):
-        e2e_step()
+    e2e_steps(2)
     torch.cuda.synchronize(dev)
-    erep = max(3, min(args.steps, 10))
+    erep = 3 if long_step else max(3, min(args.steps, 10))
     barrier()
     e0.record(stream)
-    for _ in range(erep):
-        e2e_step()
+    e2e_steps(erep)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / erep)
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
     d2h = hout.numel() * hout.element_size()
+    del bufs
 
     peaks, peak_src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sustained = float(peaks.get("bf16_tflops_sustained", burst))
+    peak, which = tensor_peak(peaks, ms * args.steps * 1e-3)
     hist_launch_ms = stage_ms["attn_history"] / n_pass
     hist_launch_flops = hist_flops / n_pass
     achieved = hist_launch_flops / (hist_launch_ms * 1e-3) / 1e12 if hist_launch_ms > 0 else 0.0
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     # the attention kernels together: history, own block (with its merge), merge
     attn_ms = stage_ms["attn_history"] + stage_ms["attn_current"] + stage_ms["merge"]
     attn_tflops = useful / (attn_ms * 1e-3) / 1e12 if attn_ms > 0 else 0.0
     traffic = profile_traffic(os.path.join(ROOT, "long_context_prefill_block_b200", "csrc",
                                            "attn_tc.cu"), w.name)
+    sb = stage_bytes(w)
+    stage_hbm = {}
+    for name, nbytes in sb.items():
+        t_ms = stage_ms[name]
+        gbs = nbytes / (t_ms * 1e-3) / 1e9 if t_ms > 0 else 0.0
+        stage_hbm[name] = {"algorithmic_bytes": nbytes, "gbs": gbs, "frac_of_hbm": gbs / hbm}
     tc_path = w.dtype == torch.bfloat16 and w.head_dim == 128 and w.block_size % 128 == 0
     # mean-pool, gate; per pass: 4 regroup kernels, history, own-block (+ merge on the SIMT path)
     launches_per_step = 2 + (6 if tc_path else 7) * n_pass
@@ -721,12 +902,26 @@ def main():
         if world > 1:
             torch.distributed.destroy_process_group()
         return
-    cpu = None
+    cpu = parity = None
     if world == 1 and not args.no_cpu_baseline and args.variant == "forced":
-        tf, nrows, dt, thr = time_oracle(w, q, k, v, cu, args.cpu_budget)
-        cpu = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-               "sample": f"{nrows} seeded (token, head) rows of {w.name} ({dt:.1f} s), "
-                         "useful FLOPs of those rows"}
+        # the oracle on the host cores, on the GPU arm's bits: host K and V
+        # (the pinned e2e copies) and only the sampled q rows
+        leg = time_oracle(w, hk, hv, cu, q_rows_from(q), args.cpu_budget)
+        cpu = {"value": leg["tflops"], "unit": "TFLOP/s", "cores": leg["threads"],
+               "kind": "oracle",
+               "sample": f"{len(leg['rows'])} seeded (token, head) rows of {w.name} "
+                         f"({leg['seconds']:.1f} s), useful FLOPs of those rows"}
+        # parity of this run's GPU forward on the same rows
+        out_c, lse_c = moba.moba_forward(q, k, v, cu_d, w.block_size, w.topk,
+                                         max_seqlen=w.max_seqlen, return_lse=True)
+        idx_c = moba.moba_gate_topk(q, k, cu_d, w.block_size, w.topk, max_seqlen=w.max_seqlen)
+        sel = torch.as_tensor(leg["rows"], device=dev)
+        got_out = out_c.reshape(-1, w.head_dim)[sel].float().cpu().numpy()
+        got_lse = lse_c.reshape(-1)[sel].cpu().numpy()
+        got_idx = idx_c.reshape(-1, w.topk)[sel].cpu().numpy()
+        del out_c, lse_c, idx_c
+        parity = parity_stats(w, leg, hk, hv, cu, got_out, got_lse, got_idx)
+    hashes = None if args.no_hash else input_hashes({"q": hq, "k": hk, "v": hv, "cu_seqlens": cu})
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -734,13 +929,17 @@ def main():
         "data": "synthetic", "config": config,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "attn_history", "peak_source": f"{peak_src} bf16 burst"},
+                     "kernel": "attn_history", "peak_source": f"{peak_src} bf16 {which}",
+                     "frac_of_burst": achieved / burst, "frac_of_sustained": achieved / sustained},
         "cpu_baseline": cpu,
         "e2e": {"value": useful * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "copies on their own streams, overlapped with the previous and next "
+                        "steps' compute (two device buffer sets)"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clock_info,
         "stage_ms": stage_ms,
+        "stage_hbm": stage_hbm,
         "useful_flop_per_step": useful,
         "gate_flop_per_step": gate_flops(w),
         "dense_causal_ms": dense_ms,
@@ -748,6 +947,9 @@ def main():
         "frac_of_peak_end_to_end": value / world / peak,
         "attn_kernels_tflops": attn_tflops,
         "attn_kernels_frac_of_peak": attn_tflops / peak,
+        "attn_kernels_frac_of_burst": attn_tflops / burst,
+        "parity": parity,
+        "input_sha256": hashes,
     }
     print(json.dumps(line), flush=True)
     if world > 1:
