@@ -112,6 +112,11 @@ MOBA_API moba_status moba_meanpool(const moba_params* p, const void* k, const in
  * (s_i = q . kbar_i, fp32); blocks after c are never chosen; ties go to the
  * lower block index. idx: int32 [T][Hq][k]. With own_block = 1 the own
  * block is a scored candidate (prefix mean) and appears only if chosen.
+ * Ranking resolution: scores are compared as fp32, except on the tensor-core
+ * path for 6 <= k <= 16 with the forced own block (bf16, d = 128, at most
+ * 256 blocks per sequence), which ranks 32-bit keys holding a score's top 24
+ * order bits: two scores within 2^-15 of each other (relative) rank by block
+ * index there, inside the 1e-4 relative near-tie band of the method.
  * Uses the workspace for kbar (and, with own_block = 1, for the own-block
  * scores: T * Hq floats). */
 MOBA_API moba_status moba_gate_topk(const moba_params* p, const void* q, const void* k,

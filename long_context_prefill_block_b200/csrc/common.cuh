@@ -137,6 +137,11 @@ cudaError_t launch_decode(const Dims& dm, int n_queries, const void* q, const vo
                           float* lse, int* status, cudaStream_t st);
 // Tensor-core gate (bf16, d = 128, at most 256 blocks per sequence).
 bool gate_tc_supported(const Dims& dm);
+// Its sorting-network form for 5 to 15 history slots and the forced own
+// block (gate_net.cu); launch_gate_tc hands such calls to it.
+bool gate_net_supported(const Dims& dm);
+cudaError_t launch_gate_net(const Dims& dm, const void* q, const float* kbar, const int32_t* cu,
+                            int32_t* idx, int* status, cudaStream_t st);
 cudaError_t launch_gate_tc(const Dims& dm, const void* q, const float* kbar, const float* own,
                            const int32_t* cu, int32_t* idx, int* status, cudaStream_t st);
 // own: with dm.prefix, the own-block scores [T][Hq] (launch_own_score); else unused.

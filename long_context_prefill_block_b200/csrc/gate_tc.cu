@@ -542,6 +542,7 @@ cudaError_t launch_impl(const Dims& dm, const void* q, const float* kbar, const 
 
 cudaError_t launch_gate_tc(const Dims& dm, const void* q, const float* kbar, const float* own,
                            const int32_t* cu, int32_t* idx, int* status, cudaStream_t st) {
+  if (gate_net_supported(dm)) return launch_gate_net(dm, q, kbar, cu, idx, status, st);
   return dm.prefix ? launch_impl<true>(dm, q, kbar, own, cu, idx, status, st)
                    : launch_impl<false>(dm, q, kbar, own, cu, idx, status, st);
 }
