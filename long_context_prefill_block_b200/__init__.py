@@ -50,6 +50,26 @@ class MobaError(RuntimeError):
 _lib = None
 
 
+def _configure(L: ctypes.CDLL) -> ctypes.CDLL:
+    P, V, Z = ctypes.POINTER(MobaParams), ctypes.c_void_p, ctypes.c_size_t
+    L.moba_num_blocks.argtypes = [P]
+    L.moba_num_blocks.restype = ctypes.c_int
+    L.moba_workspace_size.argtypes = [P]
+    L.moba_workspace_size.restype = Z
+    L.moba_meanpool.argtypes = [P, V, V, V, V]
+    L.moba_gate_topk.argtypes = [P, V, V, V, V, V, Z, V]
+    L.moba_forward.argtypes = [P, V, V, V, V, V, V, V, Z, V]
+    L.moba_forward_with_indices.argtypes = [P, V, V, V, V, V, V, V, V, Z, V]
+    L.dense_causal_forward.argtypes = [P, V, V, V, V, V, V, V]
+    L.moba_device_status.argtypes = [V, ctypes.c_int]
+    L.moba_status_string.argtypes = [ctypes.c_int]
+    L.moba_status_string.restype = ctypes.c_char_p
+    for name in ("moba_meanpool", "moba_gate_topk", "moba_forward",
+                 "moba_forward_with_indices", "dense_causal_forward", "moba_device_status"):
+        getattr(L, name).restype = ctypes.c_int
+    return L
+
+
 def lib() -> ctypes.CDLL:
     """The loaded libmoba.so (raises if it has not been built)."""
     global _lib
@@ -57,24 +77,19 @@ def lib() -> ctypes.CDLL:
         if not os.path.exists(LIB_PATH):
             raise ImportError(f"libmoba.so not built at {LIB_PATH}; run "
                               "`python -m long_context_prefill_block_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
-        P, V, Z = ctypes.POINTER(MobaParams), ctypes.c_void_p, ctypes.c_size_t
-        L.moba_num_blocks.argtypes = [P]
-        L.moba_num_blocks.restype = ctypes.c_int
-        L.moba_workspace_size.argtypes = [P]
-        L.moba_workspace_size.restype = Z
-        L.moba_meanpool.argtypes = [P, V, V, V, V]
-        L.moba_gate_topk.argtypes = [P, V, V, V, V, V, Z, V]
-        L.moba_forward.argtypes = [P, V, V, V, V, V, V, V, Z, V]
-        L.moba_forward_with_indices.argtypes = [P, V, V, V, V, V, V, V, V, Z, V]
-        L.dense_causal_forward.argtypes = [P, V, V, V, V, V, V, V]
-        L.moba_device_status.argtypes = [V, ctypes.c_int]
-        L.moba_status_string.argtypes = [ctypes.c_int]
-        L.moba_status_string.restype = ctypes.c_char_p
-        for name in ("moba_meanpool", "moba_gate_topk", "moba_forward",
-                     "moba_forward_with_indices", "dense_causal_forward", "moba_device_status"):
-            getattr(L, name).restype = ctypes.c_int
-        _lib = L
+        _lib = _configure(ctypes.CDLL(LIB_PATH))
+    return _lib
+
+
+def use_library(path: str) -> ctypes.CDLL:
+    """Route every call of this module through another build of the library
+    (the phase-trace build, libmoba_trace.so); must come before the first call."""
+    global _lib
+    if _lib is not None:
+        raise RuntimeError("the library is already loaded")
+    if not os.path.exists(path):
+        raise ImportError(f"{path} not built")
+    _lib = _configure(ctypes.CDLL(path))
     return _lib
 
 

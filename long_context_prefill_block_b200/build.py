@@ -1,6 +1,10 @@
 """Build libmoba.so in-tree: every csrc/*.cu compiled by nvcc for sm_100a.
 
-    python -m long_context_prefill_block_b200.build [--force]
+    python -m long_context_prefill_block_b200.build [--force] [--trace]
+
+--trace builds libmoba_trace.so instead: the same sources with MOBA_TRACE
+defined, which adds the phase-trace entry points of include/moba_trace.h
+(a measuring aid; the ordinary library carries none of it).
 """
 import concurrent.futures as cf
 import glob
@@ -13,6 +17,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmoba.so")
+OBJ_TRACE = os.path.join(HERE, "_build_trace")
+LIB_TRACE = os.path.join(HERE, "libmoba_trace.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -24,8 +30,8 @@ def _headers():
     return glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
 
 
-def _compile(src, force, extra):
-    obj = os.path.join(OBJ, os.path.basename(src) + ".o")
+def _compile(src, force, extra, objdir=OBJ):
+    obj = os.path.join(objdir, os.path.basename(src) + ".o")
     newest = max([os.path.getmtime(src)] + [os.path.getmtime(h) for h in _headers()])
     if not force and os.path.exists(obj) and os.path.getmtime(obj) >= newest:
         return obj, False
@@ -38,21 +44,25 @@ def _compile(src, force, extra):
     return obj, True
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    os.makedirs(OBJ, exist_ok=True)
+def build(force: bool = False, verbose_ptxas: bool = False, trace: bool = False) -> str:
+    objdir, lib = (OBJ_TRACE, LIB_TRACE) if trace else (OBJ, LIB)
+    os.makedirs(objdir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     extra = ["-Xptxas", "-v"] if verbose_ptxas else []
+    if trace:
+        extra = extra + ["-DMOBA_TRACE"]
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        results = list(ex.map(lambda s: _compile(s, force, extra), srcs))
+        results = list(ex.map(lambda s: _compile(s, force, extra, objdir), srcs))
     objs = [o for o, _ in results]
     changed = any(c for _, c in results)
-    if changed or force or not os.path.exists(LIB):
-        cmd = [NVCC, *ARCH, "-shared", "-o", LIB, *objs, "-Xcompiler", "-fPIC"]
+    if changed or force or not os.path.exists(lib):
+        cmd = [NVCC, *ARCH, "-shared", "-o", lib, *objs, "-Xcompiler", "-fPIC"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode:
             raise RuntimeError(f"link failed:\n{r.stderr}")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose_ptxas="--ptxas" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose_ptxas="--ptxas" in sys.argv,
+                trace="--trace" in sys.argv))

@@ -7,6 +7,14 @@
 
 #include "host_api.cuh"
 
+#ifdef MOBA_TRACE
+#include <mutex>
+#include <vector>
+
+#include "moba_trace.h"
+#include "trace.cuh"
+#endif
+
 namespace moba {
 // Per-device status word; kernels get its address, never the symbol.
 __device__ int g_status;
@@ -544,3 +552,43 @@ const char* moba_status_string(moba_status s) {
 }
 
 }  // extern "C"
+
+#ifdef MOBA_TRACE
+// ---- trace build only: the registry of the traced files' target setters
+namespace moba {
+namespace trace {
+namespace {
+std::mutex& registry_mu() {
+  static std::mutex mu;
+  return mu;
+}
+std::vector<cudaError_t (*)(const Target&)>& registry() {
+  static std::vector<cudaError_t (*)(const Target&)> fns;
+  return fns;
+}
+moba_status set_all(const Target& t) {
+  std::lock_guard<std::mutex> lock(registry_mu());
+  for (auto fn : registry())
+    if (fn(t) != cudaSuccess) return MOBA_ERR_CUDA;
+  return MOBA_OK;
+}
+}  // namespace
+void add_setter(cudaError_t (*fn)(const Target&)) {
+  std::lock_guard<std::mutex> lock(registry_mu());
+  registry().push_back(fn);
+}
+}  // namespace trace
+}  // namespace moba
+
+extern "C" {
+moba_status moba_trace_arm(int kernel, int cta, unsigned long long* buf, int* counts, int cap) {
+  if (!buf || !counts || cap <= 0 || cta < 0) return MOBA_ERR_INVALID_ARG;
+  if (cudaMemset(counts, 0, sizeof(int) * moba::trace::kMaxWarps) != cudaSuccess)
+    return MOBA_ERR_CUDA;
+  return moba::trace::set_all(moba::trace::Target{buf, counts, cap, cta, kernel});
+}
+moba_status moba_trace_disarm(void) {
+  return moba::trace::set_all(moba::trace::Target{nullptr, nullptr, 0, -1, 0});
+}
+}  // extern "C"
+#endif

@@ -15,9 +15,11 @@
 // Selection: the 256 threads of the selection warps take two per row (TMEM
 // lane = row); each copies its 16-column groups of the row's scores (every
 // other group) into registers at once, which frees the accumulator for the
-// next tile's MMA, and turns each score of a block i < c into a 32-bit
-// order key (sortnet.cuh: order-preserving score bits, low 8 bits = 255 - i;
-// blocks >= c get key 0). Per group a 16-key odd-even merge sort, then a
+// next tile's MMA, and turns each score of a block i < c into an fp32 order
+// key (sortnet.cuh: the score with its low 8 mantissa bits holding the
+// block index; blocks >= c get -inf), compared with float max / min, which
+// issue on the FMA pipes rather than the half-rate integer ALU pipe. Per
+// group a 16-key odd-even merge sort, then a
 // bitonic merge into the thread's running top 16; the two threads' lists
 // meet through TMEM and the first thread keeps the row's top 16. Every step
 // is a max/min network: no branch depends on the data, so the 32 rows of a
@@ -36,6 +38,7 @@
 
 #include "sortnet.cuh"
 #include "tc_ptx.cuh"
+#include "trace.cuh"
 
 namespace moba {
 namespace {
@@ -203,6 +206,11 @@ __global__ void __launch_bounds__(kThreads, 1) gate_net_kernel(const NetArgs a) 
   const int j0 = a.cpg ? (int)blockIdx.x % a.cpg : 0;
   const int jstep = a.cpg ? a.cpg : 1;
   const uint32_t quarter_lanes = (uint32_t)((warp & 3) * 32) << 16;
+  // phase trace (trace build only); event ids: loaders 1 item, 2 buffer free,
+  // 3 tile stored; MMA issuer 4 scores free, 5 tile ready, 6 issued;
+  // selection 10 scores ready, 11 scores in registers, 12 list sorted,
+  // 13 lists merged, 14 row written
+  MOBA_TRACE_STATE(trace::kGateNet);
 
   // The roles split here, at the top level, each with its own copy of the
   // group loop, so ptxas gives each role's code its own register budget.
@@ -225,6 +233,21 @@ __global__ void __launch_bounds__(kThreads, 1) gate_net_kernel(const NetArgs a) 
         const Item x = decode_item(a, cu, gi, j);
         if (!item_live(a, x)) continue;
         const int N = item_n(a, x);
+        MOBA_TRACE(1, N);
+        {
+          // the next item's rows of this thread into L2 while this item loads
+          int jn = j + jstep;
+          while (jn < a.ipg && !item_live(a, decode_item(a, cu, gi, jn))) jn += jstep;
+          if (jn < a.ipg) {
+            const Item xn = decode_item(a, cu, gi, jn);
+            if (xn.p0 + r < xn.len && item_n(a, xn) > 0)
+              for (int hh = 0; hh < nh; ++hh) {
+                const __nv_bfloat16* row = a.q + ((xn.start + xn.p0 + r) * dm.Hq + xn.h + hh) * 128;
+                prefetch_l2(row);
+                prefetch_l2(row + 64);
+              }
+          }
+        }
         // every Q tile of the item: load it, then (warp 0, lane 0) issue its
         // MMAs at once, so a later tile's buffer never waits on this warp
         for (int hh = 0; ok && N > 0 && hh < nh; ++hh, ++n_slot) {
@@ -233,35 +256,49 @@ __global__ void __launch_bounds__(kThreads, 1) gate_net_kernel(const NetArgs a) 
             ok = mbar_wait(&q_empty[b], ((n_slot >> 1) - 1) & 1, abort, status);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           }
+          MOBA_TRACE(2, hh);
           const int p = x.p0 + r;
           const bool has = p < x.len;
-          const uint4* src = reinterpret_cast<const uint4*>(
-              a.q + ((x.start + (has ? p : 0)) * dm.Hq + x.h + hh) * 128);
-          // 16 columns (32 bf16) at a time: the loader warps have few registers
+          const __nv_bfloat16* src = a.q + ((x.start + (has ? p : 0)) * dm.Hq + x.h + hh) * 128;
+          // the row in four 16-column pieces of two 32-byte loads each, one
+          // piece's loads in flight while the previous piece is stored (the
+          // loader warps have few registers)
+          uint32_t v[2][16];
+          auto load_piece = [&](int piece, uint32_t (&w)[16]) {
+            uint32_t lo[8], hi[8];
+            if (has) {
+              ldg_v8_b32(src + piece * 32, lo);
+              ldg_v8_b32(src + piece * 32 + 16, hi);
+            } else {
+#pragma unroll
+              for (int u = 0; u < 8; ++u) lo[u] = hi[u] = 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              w[u] = lo[u];
+              w[8 + u] = hi[u];
+            }
+          };
+          load_piece(0, v[0]);
 #pragma unroll
           for (int piece = 0; piece < 4; ++piece) {
-            uint32_t v[16];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const uint4 w = has ? __ldg(src + piece * 4 + u) : make_uint4(0, 0, 0, 0);
-              v[4 * u] = w.x;
-              v[4 * u + 1] = w.y;
-              v[4 * u + 2] = w.z;
-              v[4 * u + 3] = w.w;
-            }
-            tmem_st16(tmem + quarter_lanes + kQCol + b * 64 + piece * 16, v);
+            if (piece + 1 < 4) load_piece(piece + 1, v[(piece + 1) & 1]);
+            tmem_st16(tmem + quarter_lanes + kQCol + b * 64 + piece * 16, v[piece & 1]);
           }
           tmem_wait_st();
           fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive(&q_full[b]);
+          MOBA_TRACE(3, hh);
           if (warp == 0) {
             if (lane == 0) {
               // scores (+)= Q K^T with the three kbar terms; the first tile
               // of an item waits until the last item's scores were read out
               if (hh == 0 && n_item > 0)
                 ok = mbar_wait(&acc_empty, (n_item - 1) & 1, abort, status);
+              MOBA_TRACE(4, hh);
               if (ok) ok = mbar_wait(&q_full[b], (n_slot >> 1) & 1, abort, status);
+              MOBA_TRACE(5, hh);
               if (ok) {
                 fence_after_sync();
                 const uint32_t idesc = idesc_bf16(kRows, N, false, false);
@@ -276,6 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) gate_net_kernel(const NetArgs a) 
                   }
                 commit(&q_empty[b]);
                 if (hh == nh - 1) commit(&acc_full);
+                MOBA_TRACE(6, N);
               }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -315,64 +353,84 @@ __global__ void __launch_bounds__(kThreads, 1) gate_net_kernel(const NetArgs a) 
         const int c = valid ? p / dm.B : 0;
         ok = mbar_wait(&acc_full, n_item & 1, abort, status);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        MOBA_TRACE(10, (int)n_item);
         fence_after_sync();
         const int cw = __reduce_max_sync(0xffffffffu, c);  // columns any row of the warp needs
-        uint32_t key[8][16];
+        uint32_t raw[8][16];
 #pragma unroll
         for (int gq = 0; gq < 8; ++gq) {
           const int g = part + 2 * gq;
-          if (16 * g < cw) tmem_ld16(tmem + quarter_lanes + kAccCol + 16 * g, key[gq]);
+          if (16 * g < cw) tmem_ld16(tmem + quarter_lanes + kAccCol + 16 * g, raw[gq]);
         }
         tmem_wait_ld();
         // the scores are in registers: the next item's MMA may overwrite them
         fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty);
-        uint32_t list[16];
+        MOBA_TRACE(11, cw);
+        // fp32 keys compared with float max / min (sortnet.cuh)
+        float list[16];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) list[u] = 0u;
+        for (int u = 0; u < 16; ++u) list[u] = -INFINITY;
+        // groups below every row's own block need no mask
+        const int cmin = __reduce_min_sync(0xffffffffu, valid ? c : cw);
 #pragma unroll
         for (int gq = 0; gq < 8; ++gq) {
           const int g = part + 2 * gq;
           if (16 * g < cw) {
+            float key[16];
+            if (16 * g + 16 <= cmin) {
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              const int i = 16 * g + u;
-              key[gq][u] = i < c ? net::order_key(__uint_as_float(key[gq][u]), i) : 0u;
+              for (int u = 0; u < 16; ++u) key[u] = net::order_key(__uint_as_float(raw[gq][u]), 16 * g + u);
+            } else {
+#pragma unroll
+              for (int u = 0; u < 16; ++u) {
+                const int i = 16 * g + u;
+                key[u] = i < c ? net::order_key(__uint_as_float(raw[gq][u]), i) : -INFINITY;
+              }
             }
-            net::oe_sort16(key[gq]);
-            net::merge_top16(list, key[gq]);
+            net::oe_sort16(key);
+            net::merge_top16(list, key);
           }
         }
+        MOBA_TRACE(12, 0);
         // the two lists of the row meet through TMEM (two buffers by item parity)
         const uint32_t par = n_item & 1u;
         const uint32_t xcol = tmem + quarter_lanes + kXCol + par * 16;
         if (part == 1) {
-          tmem_st16(xcol, list);
+          uint32_t w[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) w[u] = __float_as_uint(list[u]);
+          tmem_st16(xcol, w);
           tmem_wait_st();
           fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive(&x_full[quarter][par]);
+          MOBA_TRACE(13, 0);
         } else {
           ok = mbar_wait(&x_full[quarter][par], (n_item >> 1) & 1, abort, status);
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
           fence_after_sync();
-          uint32_t other[16];
-          tmem_ld16(xcol, other);
+          uint32_t w[16];
+          tmem_ld16(xcol, w);
           tmem_wait_ld();
+          float other[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) other[u] = __uint_as_float(w[u]);
           net::merge_top16(list, other);
+          MOBA_TRACE(13, 0);
           if (valid) {
             // the top min(k-1, c) keys in ascending block order (descending
-            // 255 - i), then the own block c, then -1
+            // 255 - i, exact in fp32), then the own block c, then -1
             const int hsel = min(dm.topk - 1, c);
-            uint32_t sel[16];
+            float sel[16];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) sel[u] = u < hsel ? 0xFFFFFF00u | (list[u] & 0xFFu) : 0u;
+            for (int u = 0; u < 16; ++u)
+              sel[u] = u < hsel ? (float)(255 - net::key_block(list[u])) : -1.f;
             net::oe_sort16(sel);
             int v[16];
 #pragma unroll
-            for (int u = 0; u < 16; ++u)
-              v[u] = u < hsel ? net::key_block(sel[u]) : (u == hsel ? c : -1);
+            for (int u = 0; u < 16; ++u) v[u] = u < hsel ? 255 - (int)sel[u] : (u == hsel ? c : -1);
             for (int hh = 0; hh < nh; ++hh) {
               int32_t* row = a.idx + ((x.start + p) * dm.Hq + x.h + hh) * (int64_t)dm.topk;
               if (a.vec_rows) {
@@ -388,10 +446,12 @@ __global__ void __launch_bounds__(kThreads, 1) gate_net_kernel(const NetArgs a) 
             }
           }
         }
+        MOBA_TRACE(14, 0);
         ++n_item;
       }
     }
   }
+  MOBA_TRACE_END();
   if (!ok) *abort = 1;
   __syncthreads();
   if (tid == 0 && *abort) {

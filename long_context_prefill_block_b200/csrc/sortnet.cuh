@@ -1,5 +1,7 @@
-// Branch-free sorting networks on 16 unsigned 32-bit keys, in registers
-// (compile-time indices only), for the gate's top-k selection.
+// Branch-free sorting networks on 16 keys, in registers (compile-time
+// indices only), for the gate's top-k selection. Keys are 32-bit unsigned
+// integers or fp32 values (compared with float max / min; keys are never
+// NaN).
 //
 // oe_sort16: Batcher's odd-even merge sort (63 compare-exchanges),
 // descending: v[0] ends up the largest. merge_top16: given two descending
@@ -12,22 +14,29 @@
 // (0-1 principle: a network sorts every input iff it sorts every 0/1 input).
 #pragma once
 
+#include <math.h>
 #include <stdint.h>
 #include <string.h>
 
 namespace moba {
 namespace net {
 
-__host__ __device__ __forceinline__ void cx(uint32_t& a, uint32_t& b) {
-  const uint32_t hi = a > b ? a : b;
-  const uint32_t lo = a > b ? b : a;
+__host__ __device__ __forceinline__ uint32_t kmax(uint32_t a, uint32_t b) { return a > b ? a : b; }
+__host__ __device__ __forceinline__ uint32_t kmin(uint32_t a, uint32_t b) { return a > b ? b : a; }
+__host__ __device__ __forceinline__ float kmax(float a, float b) { return fmaxf(a, b); }
+__host__ __device__ __forceinline__ float kmin(float a, float b) { return fminf(a, b); }
+
+template <typename K>
+__host__ __device__ __forceinline__ void cx(K& a, K& b) {
+  const K hi = kmax(a, b);
+  const K lo = kmin(a, b);
   a = hi;
   b = lo;
 }
 
 // Merges the two sorted halves of v[LO .. LO+N) taking every R-th element.
-template <int LO, int N, int R>
-__host__ __device__ __forceinline__ void oe_merge(uint32_t (&v)[16]) {
+template <int LO, int N, int R, typename K>
+__host__ __device__ __forceinline__ void oe_merge(K (&v)[16]) {
   constexpr int M = 2 * R;
   if constexpr (M < N - 1) {
     oe_merge<LO, N, M>(v);
@@ -39,8 +48,8 @@ __host__ __device__ __forceinline__ void oe_merge(uint32_t (&v)[16]) {
   }
 }
 
-template <int LO, int N>
-__host__ __device__ __forceinline__ void oe_sort(uint32_t (&v)[16]) {
+template <int LO, int N, typename K>
+__host__ __device__ __forceinline__ void oe_sort(K (&v)[16]) {
   if constexpr (N > 1) {
     oe_sort<LO, N / 2>(v);
     oe_sort<LO + N / 2, N / 2>(v);
@@ -48,12 +57,16 @@ __host__ __device__ __forceinline__ void oe_sort(uint32_t (&v)[16]) {
   }
 }
 
-__host__ __device__ __forceinline__ void oe_sort16(uint32_t (&v)[16]) { oe_sort<0, 16>(v); }
+template <typename K>
+__host__ __device__ __forceinline__ void oe_sort16(K (&v)[16]) {
+  oe_sort<0, 16>(v);
+}
 
 // l, g sorted descending; l <- the 16 largest of l and g, descending.
-__host__ __device__ __forceinline__ void merge_top16(uint32_t (&l)[16], const uint32_t (&g)[16]) {
+template <typename K>
+__host__ __device__ __forceinline__ void merge_top16(K (&l)[16], const K (&g)[16]) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) l[i] = l[i] > g[15 - i] ? l[i] : g[15 - i];
+  for (int i = 0; i < 16; ++i) l[i] = kmax(l[i], g[15 - i]);
 #pragma unroll
   for (int s = 8; s >= 1; s >>= 1)
 #pragma unroll
@@ -71,20 +84,33 @@ __host__ __device__ __forceinline__ uint32_t float_bits(float s) {
 #endif
 }
 
-// Selection key of score s of block i (0 <= i < 256): the score's bits made
-// order-preserving as an unsigned integer (negative values inverted, the
-// sign bit set on the others; -0 first turned into +0), the lowest 8 bits
-// then replaced by 255 - i. A larger key is a larger score or, between
-// scores that agree in their top 24 order bits (within 2^-15 of each
-// other, relative; 2^-141 absolute among subnormals), the lower block. Empty slots use key 0, below every
-// finite score.
-__host__ __device__ __forceinline__ uint32_t order_key(float s, int i) {
-  const uint32_t u = float_bits(s + 0.0f);
-  const uint32_t ord = u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
-  return (ord & 0xFFFFFF00u) | (uint32_t)(255 - i);
+__host__ __device__ __forceinline__ float bits_float(uint32_t u) {
+#ifdef __CUDA_ARCH__
+  return __uint_as_float(u);
+#else
+  float s;
+  memcpy(&s, &u, sizeof s);
+  return s;
+#endif
 }
 
-__host__ __device__ __forceinline__ int key_block(uint32_t key) { return 255 - (int)(key & 0xFFu); }
+// Selection key of score s of block i (0 <= i < 256), as an fp32 value:
+// the score (-0 first turned into +0) with its lowest 8 mantissa bits
+// replaced by the block index -- 255 - i for a non-negative score, i for a
+// negative one -- so that under the float order a larger key is a larger
+// score or, between scores that agree in all but those 8 bits (within 2^-15
+// of each other, relative; 2^-141 absolute among subnormals), the lower
+// block. Empty slots use -inf, below every finite key.
+__host__ __device__ __forceinline__ float order_key(float s, int i) {
+  const uint32_t u = float_bits(s + 0.0f);
+  const uint32_t low = (u >> 31) ? (uint32_t)i : (uint32_t)(255 - i);
+  return bits_float((u & 0xFFFFFF00u) | low);
+}
+
+__host__ __device__ __forceinline__ int key_block(float key) {
+  const uint32_t u = float_bits(key);
+  return (u >> 31) ? (int)(u & 0xFFu) : 255 - (int)(u & 0xFFu);
+}
 
 }  // namespace net
 }  // namespace moba
