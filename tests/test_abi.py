@@ -12,10 +12,12 @@ import long_context_prefill_block_b200 as moba
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def declared_symbols():
+def declared_symbols(headers=None):
+    """Entry points declared in include/*.h (all headers but the trace build's
+    by default)."""
     names = []
-    for fn in os.listdir(os.path.join(ROOT, "include")):
-        if fn.endswith(".h"):
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h") and (fn in headers if headers else fn != "moba_trace.h"):
             text = open(os.path.join(ROOT, "include", fn)).read()
             names += re.findall(r"MOBA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
     return names
@@ -32,6 +34,21 @@ def test_library_exports_every_declared_symbol():
     lib = moba.lib()
     for name in declared_symbols():
         assert hasattr(lib, name), name
+
+
+def test_trace_entry_points_only_in_the_trace_build():
+    from long_context_prefill_block_b200 import build
+
+    names = declared_symbols(["moba_trace.h"])
+    assert set(names) == {"moba_trace_arm", "moba_trace_disarm"}
+    lib = moba.lib()
+    for name in names:
+        assert not hasattr(lib, name), name
+    if not os.path.exists(build.LIB_TRACE):
+        pytest.skip("trace build absent")
+    traced = ctypes.CDLL(build.LIB_TRACE)
+    for name in declared_symbols(["moba_trace.h"]) + declared_symbols():
+        assert hasattr(traced, name), name
 
 
 def params(**kw):
