@@ -29,15 +29,18 @@
 //               then per KV tile j O[h] += P_h(j) V(j) and S[h] = Q_h
 //               K(j+1)^T into the same TMEM -- tcgen05.mma operations of one
 //               thread run in issue order, so the PV has read P before the
-//               next QK^T overwrites it. The softmax warps hand P over in two
-//               halves (keys 0-63, then 64-127), so the first half's PV runs
-//               while the second half is exponentiated. Issuing blocks for
-//               about the group's execution time, hence one issuer per half;
+//               next QK^T overwrites it. The softmax warps hand P over in
+//               four quarters of 32 keys, so each quarter's PV runs while the
+//               next is exponentiated. Issuing blocks for about the group's
+//               execution time, hence one issuer per half;
 //   warp 3      Q loader: cp.async of each half's (gathered, in HIST mode)
 //               query rows into the swizzled layout the MMA reads;
 //   warps 4-7   softmax + epilogue of half 0, warps 8-11 of half 1: one query
 //               row per thread (TMEM lane = row), base-2 exponentials; O[h]
 //               is rescaled only when a row maximum grows by more than 2^8.
+//               The two halves take turns on the exponentials (shared-memory
+//               counters), so one half's PV and next QK^T run on the tensor
+//               core while the other half exponentiates.
 // The softmax warps get most of the register file (setmaxnreg): they hold a
 // whole 128-column row of S, or of O in the epilogue.
 //
@@ -48,6 +51,7 @@
 #include <mutex>
 
 #include "tc_ptx.cuh"
+#include "trace.cuh"
 
 namespace moba {
 
@@ -87,11 +91,17 @@ constexpr uint32_t kOCol = 256;
 constexpr uint32_t kIdescQK = idesc_bf16(TM, TN, false, false);  // Q, K both K-major
 constexpr uint32_t kIdescPV = idesc_bf16(TM, D, false, true);    // V is MN-major (d contiguous)
 constexpr float kRescaleLog2 = 8.f;
+// Softmax exponentials taken off the exponential unit: of every 8 column
+// pairs, this many go through ex2_poly2 on the FMA pipes.
+constexpr int kPolyOf8 = 0;
+// Whether the history and own-block kernels also make the two query halves
+// take turns on the exponentials (the dense kernel always does).
+constexpr bool kTurnsAll = true;
 
 struct Shared {
   // per query half h
   uint64_t q_full[kQBufs], q_empty[kQBufs];
-  uint64_t s_full[2], p_lo[2], p_full[2], o_full[2], o_free[2];
+  uint64_t s_full[2], p_q[2][4], o_full[2], o_free[2];
   uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
   uint64_t drain[2];
   uint32_t tmem_base;
@@ -292,8 +302,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sh.s_full[i], 1);
-      mbar_init(&sh.p_lo[i], 128);
-      mbar_init(&sh.p_full[i], 128);
+      for (int c = 0; c < 4; ++c) mbar_init(&sh.p_q[i][c], 128);
       mbar_init(&sh.o_full[i], 1);
       mbar_init(&sh.o_free[i], 128);
     }
@@ -319,6 +328,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
   const uint32_t tmem = sh.tmem_base;
   volatile int* abort = &sh.abort;
   int* status = a.status;
+  // phase trace (trace build only); event ids: TMA producer 20 K tile issued,
+  // 21 V tile issued; MMA issuers 30 unit, 31 QK issued, 32 P keys 0-63
+  // ready, 33 PV issued; Q loader 40 Q half loaded; softmax 50 S ready,
+  // 51 row max, 52 P keys 0-63 written, 53 P written, 54 O ready, 55 row
+  // written, 56 S in registers, 58 P computed
+  MOBA_TRACE_STATE(MODE == HIST ? trace::kAttnHist
+                                : (MODE == CUR ? trace::kAttnCur : trace::kAttnDense));
 
   if (warp < 4) {
     // warps 0-3 (one warp group) give registers to the softmax warps
@@ -339,11 +355,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
             tma_load_3d(sK + st * kTile, &tmk, &sh.k_full[st], 0, T.g, z);
             tma_load_3d(sK + st * kTile + kHalf, &tmk, &sh.k_full[st], 64, T.g, z);
             nk = g + 1;
+            MOBA_TRACE(20, j);
             if (u > 0 && !(ok = mbar_wait(&sh.v_empty[st], (u - 1) & 1, abort, status))) break;
             mbar_expect_tx(&sh.v_full[st], kTile);
             tma_load_3d(sV + st * kTile, &tmv, &sh.v_full[st], 0, T.g, z);
             tma_load_3d(sV + st * kTile + kHalf, &tmv, &sh.v_full[st], 64, T.g, z);
             nv = g + 1;
+            MOBA_TRACE(21, j);
           }
         }
         if (!ok || *abort) {
@@ -375,6 +393,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           if (t + (int)gridDim.x < n_tiles) Tnext = get_tile<MODE>(a, t + gridDim.x);
           if (T.skip) continue;
           const int nh = T.n[h];
+          MOBA_TRACE(30, nh);
           const uint32_t qslot = qs + (h == 1 && T.n[0] > 0 ? 1u : 0u);
           const uint32_t qb = qslot % kQBufs;
           qs += (T.n[0] > 0 ? 1u : 0u) + (T.n[1] > 0 ? 1u : 0u);
@@ -400,25 +419,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
               }
               commit(&sh.s_full[h]);
               if (j == nh - 1) commit(&sh.q_empty[qb]);
+              MOBA_TRACE(31, j);
             }
             commit(&sh.k_empty[st]);
-            if (j < nh) {
-              // O[h] += P_h(j) V(j), P read from the first 64 columns of S[h]
-              if (j == 0 && uh > 0 &&
-                  !(ok = mbar_wait(&sh.o_free[h], (uh - 1) & 1, abort, status)))
-                break;
-              if (!(ok = mbar_wait(&sh.p_lo[h], (kh + j) & 1, abort, status))) break;
-            }
+            if (j < nh && j == 0 && uh > 0 &&
+                !(ok = mbar_wait(&sh.o_free[h], (uh - 1) & 1, abort, status)))
+              break;
             if (!(ok = mbar_wait(&sh.v_full[st], (gg / NS) & 1, abort, status))) break;
             if (j < nh) {
-              // keys 0-63 of P are written first: their PV runs while the
-              // softmax warps still exponentiate keys 64-127
-              fence_after_sync();
+              // O[h] += P_h(j) V(j), P read from the first 64 columns of S[h].
+              // P arrives in quarters of 32 keys (two k-steps each): each
+              // quarter's PV runs while the softmax warps exponentiate the next
 #pragma unroll
               for (int kk = 0; kk < TN / 16; ++kk) {
-                if (kk == TN / 32) {
-                  if (!(ok = mbar_wait(&sh.p_full[h], (kh + j) & 1, abort, status))) break;
+                if ((kk & 1) == 0) {
+                  if (!(ok = mbar_wait(&sh.p_q[h][kk >> 1], (kh + j) & 1, abort, status))) break;
                   fence_after_sync();
+                  if (kk == 0) MOBA_TRACE(32, j);
                 }
                 const uint64_t bd = desc_sw128(sV + st * kTile + kk * 16 * 128, kHalf, 1024);
                 mma_ts(tmem + kOCol + h * 128, tmem + h * 128 + kk * 8, bd, kIdescPV,
@@ -426,6 +443,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
               }
               if (!ok) break;
               if (j == nh - 1) commit(&sh.o_full[h]);
+              MOBA_TRACE(33, j);
             }
             commit(&sh.v_empty[st]);
           }
@@ -498,6 +516,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           cp_async_wait_all();
           fence_proxy_async_smem();
           mbar_arrive(&sh.q_full[qb]);
+          MOBA_TRACE(40, h);
           ++qs;
         }
         if (!ok) break;
@@ -538,6 +557,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
       for (int j = 0; j < T.n_kv; ++j, ++kc) {
         ok = mbar_wait(&sh.s_full[hh], kc & 1, abort, status);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        MOBA_TRACE(50, j);
         fence_after_sync();
         float s[TN];
         {
@@ -548,6 +568,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           tmem_ld32(tS + 64, r2);
           tmem_ld32(tS + 96, r3);
           tmem_wait_ld();
+          MOBA_TRACE(56, j);
 #pragma unroll
           for (int x = 0; x < 32; ++x) {
             s[x] = __uint_as_float(r0[x]);
@@ -563,17 +584,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           for (int x = 0; x < TN; ++x)
             if (x > lim) s[x] = -INFINITY;
         }
-        // row maximum as a tree of 8 independent chains
-        float mv[8];
+        // row maximum: 16 independent chains of three-input maxima (chain u
+        // takes columns u, u + 16, ..., u + 112: four instructions deep),
+        // then a three-input tree
+        float mv[16];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) mv[u] = s[u];
+        for (int u = 0; u < 16; ++u) {
+          const float a = fmax3(s[u], s[u + 16], s[u + 32]);
+          const float b = fmax3(a, s[u + 48], s[u + 64]);
+          const float c = fmax3(b, s[u + 80], s[u + 96]);
+          mv[u] = fmaxf(c, s[u + 112]);
+        }
+        float m6[6];
 #pragma unroll
-        for (int x = 8; x < TN; x += 8)
-#pragma unroll
-          for (int u = 0; u < 8; ++u) mv[u] = fmaxf(mv[u], s[x + u]);
-        const float mx = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
-                               fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
+        for (int u = 0; u < 5; ++u) m6[u] = fmax3(mv[3 * u], mv[3 * u + 1], mv[3 * u + 2]);
+        m6[5] = mv[15];
+        const float mx = fmax3(fmax3(m6[0], m6[1], m6[2]), fmax3(m6[3], m6[4], m6[5]), m6[0]);
         const float mt = mx * sl2;
+        MOBA_TRACE(51, j);
         const bool need = mt > m_i + kRescaleLog2;
         const float m_new = need ? mt : m_i;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
@@ -595,16 +623,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           l_i *= ex2(m_i - m_new);
           m_i = m_new;
         }
-        // DENSE: the two halves take turns on the exponential unit: half 1
+        // The two halves take turns on the exponential unit: half 1
         // exponentiates KV tile j after half 0 has, half 0 tile j after half
         // 1 has done tile j - 1. In anti-phase, one half's PV and next QK^T
-        // run while the other half exponentiates. (HIST and CUR units are
-        // only a few KV tiles long and run faster without the turns: one
-        // warp per SM sub-partition reaches only about half the exponential
-        // rate of two.)
+        // run while the other half exponentiates (measured: history 870 ->
+        // 809 ms at the million-token shape, 0.80 -> 0.75 ms at 32K).
         // Counts only grow, so a half that runs ahead into its next unit
         // cannot be mistaken for the turn being waited for.
-        if (MODE == DENSE && (hh == 0 ? (j >= 1 && j - 1 < T0.n[1]) : (j < T0.n[0]))) {
+        if ((MODE == DENSE || kTurnsAll) &&
+            (hh == 0 ? (j >= 1 && j - 1 < T0.n[1]) : (j < T0.n[0]))) {
           const int need_cnt = 4 * (hh == 0 ? b1 + j : b0 + j + 1);
           const long long t0 = clock64();
           while (exp_cnt[hh ^ 1] < need_cnt) {
@@ -618,36 +645,57 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           }
           if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         }
-        // P = exp2(s * scale - m) in bf16, two per column, into the S buffer;
-        // the row sum is kept in 8 independent partial sums
-        float ps[8];
+        // P = exp2(s * scale - m) in bf16, two per column, into the S buffer,
+        // on column pairs (f32x2): kPolyOf8 of every 8 pairs by ex2_poly2 on
+        // the FMA pipes, the others on the exponential unit; the row sum is
+        // kept in 4 independent pair sums. P goes to the MMA issuer in four
+        // quarters of 32 keys: quarter c is stored once computed, and waited
+        // for (tcgen05.wait::st covers every earlier store) only after quarter
+        // c + 1 is computed, so only the last store's latency is exposed.
+        const uint64_t sl2x2 = f2(sl2, sl2), negm2 = f2(-m_i, -m_i);
+        uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};  // +0.f pairs
+        uint32_t pk[2][16];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) ps[u] = 0.f;
+        for (int c = 0; c < 4; ++c) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const float e0 = ex2(fmaf(s[c * 64 + 2 * x], sl2, -m_i));
-            const float e1 = ex2(fmaf(s[c * 64 + 2 * x + 1], sl2, -m_i));
-            ps[(2 * x) & 7] += e0;
-            ps[(2 * x + 1) & 7] += e1;
-            pk[x] = pack_bf16x2(e0, e1);
+          for (int x = 0; x < 16; ++x) {
+            const int col = c * 32 + 2 * x;
+            const uint64_t a2 = ffma2(f2(s[col], s[col + 1]), sl2x2, negm2);
+            uint64_t e2;
+            if (x % 8 < kPolyOf8) {
+              e2 = ex2_poly2(a2);
+            } else {
+              float a0, a1;
+              f2split(a2, a0, a1);
+              e2 = f2(ex2(a0), ex2(a1));
+            }
+            ps2[x & 3] = fadd2(ps2[x & 3], e2);
+            float e0, e1;
+            f2split(e2, e0, e1);
+            pk[c & 1][x] = pack_bf16x2(e0, e1);
           }
-          tmem_st32(tS + c * 32, pk);
-          if (c == 0) {
-            // keys 0-63 of P are in TMEM: their PV may start
+          if (c > 0) {
+            // quarter c - 1 is in TMEM: its PV may start
             tmem_wait_st();
             fence_before_sync();
-            mbar_arrive(&sh.p_lo[hh]);
+            mbar_arrive(&sh.p_q[hh][c - 1]);
+            if (c == 2) MOBA_TRACE(52, j);
           }
+          tmem_st16(tS + c * 16, pk[c & 1]);
         }
+        MOBA_TRACE(58, j);
         __syncwarp();
         if (lane == 0) atomicAdd(const_cast<int*>(&exp_cnt[hh]), 1);
         tmem_wait_st();
-        l_i += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        {
+          const uint64_t q2 = fadd2(fadd2(ps2[0], ps2[1]), fadd2(ps2[2], ps2[3]));
+          float q0, q1;
+          f2split(q2, q0, q1);
+          l_i += q0 + q1;
+        }
         fence_before_sync();
-        mbar_arrive(&sh.p_full[hh]);
+        mbar_arrive(&sh.p_q[hh][3]);
+        MOBA_TRACE(53, j);
       }
       if (!ok) break;
       // ---- epilogue: wait for the half's last PV, normalise, write
@@ -682,6 +730,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
       }
       ok = mbar_wait(&sh.o_full[hh], uc & 1, abort, status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      MOBA_TRACE(54, 0);
       fence_after_sync();
       if (MODE == CUR) {
         // Own block done: merge with this row's history partials right here
@@ -813,9 +862,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
           }
         }
       }
+      MOBA_TRACE(55, 0);
       ++uc;
     }
   }
+  MOBA_TRACE_END();
 
   fence_before_sync();
   __syncthreads();

@@ -247,6 +247,65 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// max of three (sm_100 three-input max.f32): half the instructions of a
+// two-input max tree
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// ---- packed fp32 pairs (sm_100 f32x2): one instruction for two lanes of work
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^x of a pair without the exponential unit (the softmax's busier unit),
+// on the FMA pipes: Cody-Waite range reduction x = j + f with j = round(x)
+// -- adding and subtracting 1.5 * 2^23 rounds to an integer, whose value
+// the low bits of the sum then hold -- and |f| <= 1/2; 2^f by the degree-3
+// polynomial minimising the relative error on [-1/2, 1/2] (Lawson's
+// reweighted least squares, fit_exp2.py; max relative error 7.5e-5 in fp32,
+// far below the bf16 rounding of P); 2^j enters as an integer add to the
+// exponent field. x is first clamped at -125 so that field stays positive:
+// a masked score (-inf) then weighs 2^-125 (about 2e-38), not 0.
+__device__ __forceinline__ uint64_t ex2_poly2(uint64_t x) {
+  float x0, x1;
+  f2split(x, x0, x1);
+  const uint64_t xc = f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t round2 = f2(12582912.f, 12582912.f);  // 1.5 * 2^23
+  const uint64_t t = fadd2(xc, round2);
+  const uint64_t f = fsub2(xc, fsub2(t, round2));
+  uint64_t p = ffma2(f, f2(0.0551716685f, 0.0551716685f), f2(0.242611125f, 0.242611125f));
+  p = ffma2(p, f, f2(0.693260968f, 0.693260968f));
+  p = ffma2(p, f, f2(0.999928057f, 0.999928057f));
+  float p0, p1, t0, t1;
+  f2split(p, p0, p1);
+  f2split(t, t0, t1);
+  return f2(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+            __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

@@ -38,8 +38,12 @@ EVENTS = {
     "gate": {1: "item", 2: "q buffer free", 3: "q tile stored", 4: "scores free",
              5: "q tile ready", 6: "mma issued", 10: "scores ready", 11: "scores in regs",
              12: "list sorted", 13: "lists merged", 14: "row written"},
-    "hist": {}, "cur": {}, "dense": {},
 }
+EVENTS["hist"] = EVENTS["cur"] = EVENTS["dense"] = {
+    20: "K issued", 21: "V issued", 30: "unit", 31: "QK issued", 32: "P lo ready",
+    33: "PV issued", 40: "Q half loaded", 50: "S ready", 51: "row max", 52: "P lo written",
+    53: "P written", 54: "O ready", 55: "row written", 56: "S in regs", 57: "P lo computed",
+    58: "P hi computed"}
 
 
 def run(workload: str, kernel: str, cta: int, cap: int, mhz: float, shared: bool):
