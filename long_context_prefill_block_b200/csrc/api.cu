@@ -138,7 +138,7 @@ Layout plan(const Dims& dm, bool own_idx) {
   L.list_off = take(sizeof(int32_t) * (n_lists + 1));
   L.tile_off = take(sizeof(int32_t) * (n_lists + 1));
   L.pairs = take(sizeof(int32_t) * max_pairs);
-  L.tiles = take(sizeof(int2) * L.max_tiles);
+  L.tiles = take(sizeof(int4) * L.max_tiles);
   const size_t prows = part_rows(dm.T, (int64_t)L.ng * grp * dm.topk);
   L.part_o = take((dm.dtype == kBF16 ? 2 : 4) * prows * dm.d);
   L.part_lse = take(sizeof(float) * prows);
@@ -210,7 +210,7 @@ moba_status forward_impl(const moba_params* p, const void* q, const void* k, con
   rg.list_off = reinterpret_cast<int32_t*>(base + L.list_off);
   rg.tile_off = reinterpret_cast<int32_t*>(base + L.tile_off);
   rg.pairs = reinterpret_cast<int32_t*>(base + L.pairs);
-  rg.tiles = reinterpret_cast<int2*>(base + L.tiles);
+  rg.tiles = reinterpret_cast<int4*>(base + L.tiles);
   Partials pt{base + L.part_o, reinterpret_cast<float*>(base + L.part_lse)};
   for (int g0 = 0; g0 < dm.Hkv; g0 += L.ng) {
     Chunk ch;
@@ -268,7 +268,7 @@ BwdLayout plan_bwd(const Dims& dm, bool own_idx) {
   L.list_off = take(sizeof(int32_t) * (n_lists + 1));
   L.tile_off = take(sizeof(int32_t) * (n_lists + 1));
   L.pairs = take(sizeof(int32_t) * max_pairs);
-  L.tiles = take(sizeof(int2) * L.max_tiles);
+  L.tiles = take(sizeof(int4) * L.max_tiles);
   L.dsum = take(sizeof(float) * (size_t)dm.T * dm.Hq);
   L.total = off;
   return L;
@@ -309,7 +309,7 @@ moba_status backward_impl(const moba_params* p, const void* q, const void* k, co
   rg.list_off = reinterpret_cast<int32_t*>(base + L.list_off);
   rg.tile_off = reinterpret_cast<int32_t*>(base + L.tile_off);
   rg.pairs = reinterpret_cast<int32_t*>(base + L.pairs);
-  rg.tiles = reinterpret_cast<int2*>(base + L.tiles);
+  rg.tiles = reinterpret_cast<int4*>(base + L.tiles);
   rg.max_tiles = L.max_tiles;
   Chunk ch;
   ch.g0 = 0;

@@ -31,7 +31,7 @@ __global__ void __launch_bounds__(kThreads)
 attn_simt(Dims dm, Chunk ch, const T* __restrict__ q, const T* __restrict__ k,
           const T* __restrict__ v, const int32_t* __restrict__ cu,
           const int32_t* __restrict__ list_off, const int32_t* __restrict__ pairs,
-          const int2* __restrict__ tiles, const int32_t* __restrict__ tile_count,
+          const int4* __restrict__ tiles, const int32_t* __restrict__ tile_count,
           const int32_t* __restrict__ idx, void* __restrict__ part_o,
           float* __restrict__ part_lse, T* __restrict__ out, float* __restrict__ lse_out) {
   __shared__ __align__(16) float ks[kKC][D + 4];
@@ -48,17 +48,17 @@ attn_simt(Dims dm, Chunk ch, const T* __restrict__ q, const T* __restrict__ k,
 
   if (MODE == HIST) {
     if ((int)blockIdx.x >= *tile_count) return;
-    const int2 tl = tiles[blockIdx.x];
+    const int4 tl = tiles[blockIdx.x];
     const int L = tl.x;
     const int e = L % dm.nb;
     const int gl = (L / dm.nb) % ch.ng;
     b = L / (dm.nb * ch.ng);
     g = ch.g0 + gl;
-    const int count = list_off[L + 1] - list_off[L];
+    const int count = tl.z;
     const int r = tl.y + rloc;
     valid = r < count;
     if (valid) {
-      prow = pairs[list_off[L] + r];
+      prow = pairs[tl.w + r];
       const int64_t th = prow / dm.topk;
       t = th / ch.nq;
       h = ch.h0 + (int)(th % ch.nq);

@@ -86,6 +86,7 @@ constexpr uint32_t kQOff = 0;                // Q[kQBufs]
 constexpr uint32_t kKOff = kQBufs * kTile;   // K[NS]
 constexpr uint32_t kVOff = kKOff + NS * kTile;
 constexpr uint32_t kSmemBytes = kVOff + NS * kTile + 1024;  // + 1024-byte alignment slack
+constexpr int kCuSmem = 257;  // sequence offsets kept in shared memory
 constexpr uint32_t kTmemCols = 512;    // S[0] 0, S[1] 128, O[0] 256, O[1] 384
 constexpr uint32_t kOCol = 256;
 constexpr uint32_t kIdescQK = idesc_bf16(TM, TN, false, false);  // Q, K both K-major
@@ -107,6 +108,7 @@ struct Shared {
   uint32_t tmem_base;
   int abort;
   int exp_cnt[2];  // per half: softmax warps done with a KV tile's exponentials
+  int32_t cu[kCuSmem];  // sequence offsets (batch < kCuSmem), read without global loads
 };
 
 struct Args {
@@ -118,7 +120,7 @@ struct Args {
   // HIST
   const int32_t* list_off;
   const int32_t* pairs;
-  const int2* tiles;
+  const int4* tiles;
   const int32_t* tile_count;
   // CUR
   const int32_t* idx;
@@ -135,31 +137,24 @@ struct Args {
 // the unit streams max(n[0], n[1]) KV tiles.
 struct Tile {
   bool skip;
-  int b, g, h, kv0, n_kv, p0, list, row0, count;
+  int b, g, h, kv0, n_kv, p0, list, row0, count, base;
   int n[2];
   int64_t start;
+  int4 raw;  // HIST: the tile-table entry, decoded by resolve()
 };
 
 // Unit t of the static unit space. CUR / DENSE units are ordered longest
-// first so the persistent CTAs end together.
+// first so the persistent CTAs end together. A HIST unit is one 16-byte
+// load of the tile table, decoded later by resolve(): the roles fetch the
+// next unit's description a unit ahead, and the load must not stall them
+// until the unit starts.
 template <int MODE>
-__device__ __forceinline__ Tile get_tile(const Args& a, int t) {
+__device__ __forceinline__ Tile get_tile(const Args& a, const int32_t* cu, int t) {
   const Dims& dm = a.dm;
   Tile T{};
   T.skip = false;
   if (MODE == HIST) {
-    const int2 tl = a.tiles[t];
-    T.list = tl.x;
-    T.row0 = tl.y;
-    const int e = T.list % dm.nb;
-    T.g = a.ch.g0 + (T.list / dm.nb) % a.ch.ng;
-    T.b = T.list / (dm.nb * a.ch.ng);
-    T.count = a.list_off[T.list + 1] - a.list_off[T.list];
-    T.kv0 = e * dm.B;
-    T.n_kv = dm.B / TN;
-    T.n[0] = T.n_kv;
-    T.n[1] = T.row0 + TM < T.count ? T.n_kv : 0;
-    T.start = a.cu[T.b];
+    T.raw = a.tiles[t];  // list, first row, list size, list base
     return T;
   }
   int m;  // the unit holds query tiles 2m and 2m + 1 (of the block / sequence)
@@ -190,12 +185,34 @@ __device__ __forceinline__ Tile get_tile(const Args& a, int t) {
   }
   T.n[0] = 2 * m + 1;
   T.g = T.h / (dm.Hq / dm.Hkv);
-  T.start = a.cu[T.b];
-  const int len = a.cu[T.b + 1] - a.cu[T.b];
+  T.start = cu[T.b];
+  const int len = cu[T.b + 1] - cu[T.b];
   T.count = len;  // sequence length, for the row checks below
   T.skip = len < 0 || len > dm.max_seqlen || T.p0 >= len;
   if (T.p0 + TM >= len) T.n[1] = 0;
   T.n_kv = T.n[1] > T.n[0] ? T.n[1] : T.n[0];
+  return T;
+}
+
+// Decodes a HIST unit's tile-table entry (CUR / DENSE units are complete).
+template <int MODE>
+__device__ __forceinline__ Tile resolve(const Args& a, const int32_t* cu, Tile T) {
+  if (MODE == HIST) {
+    const Dims& dm = a.dm;
+    const int4 tl = T.raw;
+    T.list = tl.x;
+    T.row0 = tl.y;
+    const int e = T.list % dm.nb;
+    T.g = a.ch.g0 + (T.list / dm.nb) % a.ch.ng;
+    T.b = T.list / (dm.nb * a.ch.ng);
+    T.count = tl.z;
+    T.base = tl.w;
+    T.kv0 = e * dm.B;
+    T.n_kv = dm.B / TN;
+    T.n[0] = T.n_kv;
+    T.n[1] = T.row0 + TM < T.count ? T.n_kv : 0;
+    T.start = cu[T.b];
+  }
   return T;
 }
 
@@ -230,7 +247,7 @@ __device__ __forceinline__ Row get_row(const Args& a, const Tile& T, int r) {
   if (MODE == HIST) {
     R.has_q = R.valid = T.row0 + r < T.count;
     if (R.valid) {
-      R.prow = a.pairs[a.list_off[T.list] + T.row0 + r];
+      R.prow = a.pairs[T.base + T.row0 + r];
       const int64_t th = R.prow / dm.topk;
       R.t = th / a.ch.nq;
       R.h = a.ch.h0 + (int)(th % a.ch.nq);
@@ -262,7 +279,7 @@ template <int MODE>
 __device__ __forceinline__ bool q_row_of(const Args& a, const Tile& T, int r, int64_t& qrow) {
   if (MODE == HIST) {
     if (T.row0 + r >= T.count) return false;
-    const int64_t prow = a.pairs[a.list_off[T.list] + T.row0 + r];
+    const int64_t prow = a.pairs[T.base + T.row0 + r];
     const int64_t th = prow / a.dm.topk;
     qrow = (th / a.ch.nq) * a.dm.Hq + a.ch.h0 + (int)(th % a.ch.nq);
     return true;
@@ -295,6 +312,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sQ = sbase + kQOff, sK = sbase + kKOff, sV = sbase + kVOff;
 
+  const bool cu_in_smem = dm.batch < kCuSmem;
+  if (cu_in_smem)
+    for (int i = threadIdx.x; i <= dm.batch; i += kThreads) sh.cu[i] = a.cu[i];
+  const int32_t* cuv = cu_in_smem ? sh.cu : a.cu;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kQBufs; ++i) {
       mbar_init(&sh.q_full[i], kLoaderThreads);
@@ -344,8 +365,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
       if (lane == 0) {
         uint32_t g = 0, nk = 0, nv = 0;
         bool ok = true;
+        Tile Tnext = (int)blockIdx.x < n_tiles ? get_tile<MODE>(a, cuv, blockIdx.x) : Tile{};
         for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-          const Tile T = get_tile<MODE>(a, t);
+          const Tile T = resolve<MODE>(a, cuv, Tnext);  // read one unit ahead
+          if (t + (int)gridDim.x < n_tiles) Tnext = get_tile<MODE>(a, cuv, t + gridDim.x);
           if (T.skip) continue;
           for (int j = 0; j < T.n_kv; ++j, ++g) {
             const uint32_t st = g % NS, u = g / NS;
@@ -387,10 +410,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
         uint32_t uh = 0;  // units with this half non-empty before this one
         uint32_t qs = 0;  // Q slots (loads of either half) before this unit
         bool ok = true;
-        Tile Tnext = (int)blockIdx.x < n_tiles ? get_tile<MODE>(a, blockIdx.x) : Tile{};
+        Tile Tnext = (int)blockIdx.x < n_tiles ? get_tile<MODE>(a, cuv, blockIdx.x) : Tile{};
         for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-          const Tile T = Tnext;  // read one unit ahead
-          if (t + (int)gridDim.x < n_tiles) Tnext = get_tile<MODE>(a, t + gridDim.x);
+          const Tile T = resolve<MODE>(a, cuv, Tnext);  // read one unit ahead
+          if (t + (int)gridDim.x < n_tiles) Tnext = get_tile<MODE>(a, cuv, t + gridDim.x);
           if (T.skip) continue;
           const int nh = T.n[h];
           MOBA_TRACE(30, nh);
@@ -469,13 +492,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
       bool ok = true;
       auto next_unit = [&](int t) {
         for (; t < n_tiles; t += gridDim.x)
-          if (!get_tile<MODE>(a, t).skip) break;
+          if (!get_tile<MODE>(a, cuv, t).skip) break;
         return t;
       };
       // row ids (t * Hq + h < 2^31, checked on the host) of both halves of
       // unit t, -1 where a row is empty; bit h of the result: half h reads
       auto fetch_rows = [&](int t, int32_t (&qr)[2][RPL]) {
-        const Tile T = get_tile<MODE>(a, t);
+        const Tile T = resolve<MODE>(a, cuv, get_tile<MODE>(a, cuv, t));
         int mask = 0;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -542,10 +565,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
     bool ok = true;
     // the unit's description is read one unit ahead: its global loads (tile
     // table, list offsets, sequence bounds) resolve while this unit runs
-    Tile Tnext = (int)blockIdx.x < n_tiles ? get_tile<MODE>(a, blockIdx.x) : Tile{};
+    Tile Tnext = (int)blockIdx.x < n_tiles ? get_tile<MODE>(a, cuv, blockIdx.x) : Tile{};
     for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
-      const Tile T0 = Tnext;
-      if (t + (int)gridDim.x < n_tiles) Tnext = get_tile<MODE>(a, t + gridDim.x);
+      const Tile T0 = resolve<MODE>(a, cuv, Tnext);
+      if (t + (int)gridDim.x < n_tiles) Tnext = get_tile<MODE>(a, cuv, t + gridDim.x);
       if (T0.skip) continue;
       const int b0 = base[0], b1 = base[1];
       base[0] += T0.n[0];

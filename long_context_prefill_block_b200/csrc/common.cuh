@@ -159,7 +159,8 @@ struct Regroup {
   int32_t* list_off;   // [n_lists + 1]
   int32_t* tile_off;   // [n_lists + 1]; tile_off[n_lists] = number of tiles
   int32_t* pairs;      // [max pairs] partial-row ids grouped by list
-  int2* tiles;         // [max tiles] (list, first row in list)
+  int4* tiles;         // [max tiles] (list, first row in list, list size, list's first entry):
+                       // a work unit's description in one 16-byte load
   int64_t max_tiles;
 };
 cudaError_t launch_regroup(const Dims& dm, const Chunk& ch, const int32_t* idx, const int32_t* cu,

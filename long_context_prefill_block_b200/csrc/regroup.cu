@@ -51,6 +51,33 @@ __device__ __forceinline__ bool walk_row(const int32_t* row, int topk, int c, bo
   return ok && (seen_c || (!own_required && prev >= 0));
 }
 
+// walk_row over a row held in registers (k <= 32), unrolled so that every
+// index is a compile-time constant and the row stays in registers.
+template <typename F>
+__device__ __forceinline__ bool walk_row(const int32_t (&row)[32], int topk, int c,
+                                         bool own_required, F f) {
+  int prev = -1;
+  bool seen_c = false, seen_pad = false, ok = true;
+#pragma unroll
+  for (int r = 0; r < 32; ++r) {
+    if (r >= topk) break;
+    const int e = row[r];
+    if (seen_c || seen_pad) {
+      ok &= (e == -1);
+    } else if (e == c) {
+      seen_c = true;
+    } else if (e == -1) {
+      seen_pad = true;
+    } else if (e >= 0 && e < c && e > prev) {
+      prev = e;
+      f(r, e);
+    } else {
+      ok = false;
+    }
+  }
+  return ok && (seen_c || (!own_required && prev >= 0));
+}
+
 template <bool SCATTER>
 __global__ void __launch_bounds__(kThreads) regroup_pass(Dims dm, Chunk ch,
                                                          const int32_t* __restrict__ idx,
@@ -98,7 +125,7 @@ __global__ void __launch_bounds__(kRows) regroup_pass_smem(Dims dm, Chunk ch,
                                                            const int32_t* __restrict__ cu,
                                                            int32_t* counts, int32_t* cursor,
                                                            const int32_t* __restrict__ list_off,
-                                                           int32_t* pairs, int* status) {
+                                                           int32_t* pairs, int* status, int vec) {
   extern __shared__ int32_t lsm[];
   int32_t* hist = lsm;            // [nb] entries of this CTA per block
   int32_t* base = lsm + dm.nb;    // [nb] SCATTER: first list position reserved for the CTA
@@ -118,7 +145,20 @@ __global__ void __launch_bounds__(kRows) regroup_pass_smem(Dims dm, Chunk ch,
   const bool valid = p < len;
   const int64_t t = start + p;
   const int c = p / dm.B;
-  const int32_t* row = idx + (t * dm.Hq + h) * (int64_t)dm.topk;
+  const int32_t* row_g = idx + (t * dm.Hq + h) * (int64_t)dm.topk;
+  // the row in registers, by 16-byte loads when its length allows
+  int32_t row[32];
+  if (valid) {
+    if (vec) {
+#pragma unroll
+      for (int r = 0; r < 32; r += 4)
+        if (r < dm.topk) *reinterpret_cast<int4*>(row + r) = *reinterpret_cast<const int4*>(row_g + r);
+    } else {
+#pragma unroll
+      for (int r = 0; r < 32; ++r)
+        if (r < dm.topk) row[r] = row_g[r];
+    }
+  }
   const int list0 = (b * ch.ng + gl) * dm.nb;
   const int64_t prow0 = (t * ch.nq + hl) * (int64_t)dm.topk;
   bool ok = true;
@@ -208,14 +248,21 @@ __global__ void __launch_bounds__(kScanThreads) regroup_scan(int n_lists, int ti
   }
 }
 
-// Tile table: tile j of list L covers list rows [j * tile_m, (j+1) * tile_m).
+// Tile table: tile j of list L covers list rows [j * tile_m, (j+1) * tile_m);
+// each entry also carries the list's size and first entry, so a work unit's
+// description is one 16-byte load with no dependent loads behind it.
+// One CTA per list, its threads writing consecutive entries (a list of the
+// million-token shape holds hundreds of tiles).
 __global__ void regroup_tiles(int n_lists, int tile_m, const int32_t* __restrict__ counts,
-                              const int32_t* __restrict__ tile_off, int2* tiles) {
-  const int L = blockIdx.x * blockDim.x + threadIdx.x;
+                              const int32_t* __restrict__ list_off,
+                              const int32_t* __restrict__ tile_off, int4* tiles) {
+  const int L = blockIdx.x;
   if (L >= n_lists) return;
-  const int n = (counts[L] + tile_m - 1) / tile_m;
-  const int o = tile_off[L];
-  for (int j = 0; j < n; ++j) tiles[o + j] = make_int2(L, j * tile_m);
+  const int count = counts[L];
+  const int n = (count + tile_m - 1) / tile_m;
+  const int o = tile_off[L], first = list_off[L];
+  for (int j = threadIdx.x; j < n; j += blockDim.x)
+    tiles[o + j] = make_int4(L, j * tile_m, count, first);
 }
 
 }  // namespace
@@ -228,6 +275,8 @@ cudaError_t launch_regroup(const Dims& dm, const Chunk& ch, const int32_t* idx, 
     return cudaMemsetAsync(rg.tile_off + ch.n_lists, 0, sizeof(int32_t), st);
   }
   const bool smem_lists = dm.nb <= kSmemLists;
+  // index rows start on 16-byte boundaries when k % 4 == 0 and idx does
+  const int vec = (dm.topk % 4 == 0 && (reinterpret_cast<uintptr_t>(idx) & 15) == 0) ? 1 : 0;
   dim3 grid((dm.max_seqlen + kThreads - 1) / kThreads, dm.batch, ch.nq);
   dim3 grid_s((dm.max_seqlen + kRows - 1) / kRows, dm.batch, ch.nq);
   const size_t lsm = 2 * sizeof(int32_t) * dm.nb;
@@ -239,7 +288,7 @@ cudaError_t launch_regroup(const Dims& dm, const Chunk& ch, const int32_t* idx, 
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lsm)))
       return e;
     regroup_pass_smem<false><<<grid_s, kRows, lsm, st>>>(dm, ch, idx, cu, rg.counts, rg.cursor,
-                                                         nullptr, nullptr, status);
+                                                         nullptr, nullptr, status, vec);
   } else {
     regroup_pass<false><<<grid, kThreads, 0, st>>>(dm, ch, idx, cu, rg.counts, rg.cursor, nullptr,
                                                    nullptr, status);
@@ -251,14 +300,14 @@ cudaError_t launch_regroup(const Dims& dm, const Chunk& ch, const int32_t* idx, 
   if ((e = cudaGetLastError())) return e;
   if (smem_lists) {
     regroup_pass_smem<true><<<grid_s, kRows, lsm, st>>>(dm, ch, idx, cu, rg.counts, rg.cursor,
-                                                        rg.list_off, rg.pairs, status);
+                                                        rg.list_off, rg.pairs, status, vec);
   } else {
     regroup_pass<true><<<grid, kThreads, 0, st>>>(dm, ch, idx, cu, rg.counts, rg.cursor,
                                                   rg.list_off, rg.pairs, status);
   }
   if ((e = cudaGetLastError())) return e;
-  regroup_tiles<<<(ch.n_lists + 255) / 256, 256, 0, st>>>(ch.n_lists, ch.tile_m, rg.counts,
-                                                          rg.tile_off, rg.tiles);
+  regroup_tiles<<<ch.n_lists, 128, 0, st>>>(ch.n_lists, ch.tile_m, rg.counts, rg.list_off,
+                                            rg.tile_off, rg.tiles);
   return cudaGetLastError();
 }
 
