@@ -56,7 +56,10 @@ typedef enum {
   MOBA_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed */
   MOBA_ERR_TIMEOUT = -4,      /* a bounded device wait expired */
   MOBA_ERR_WORKSPACE = -5,    /* workspace null or smaller than moba_workspace_size() */
-  MOBA_ERR_BAD_INDICES = -6   /* an index row was not in canonical form */
+  MOBA_ERR_BAD_INDICES = -6,  /* an index row was not in canonical form */
+  MOBA_ERR_CHECK = -7         /* checked build only (libmoba_checked.so, built with
+                                 MOBA_CHECKED): a device index or bounds check failed;
+                                 the access was skipped */
 } moba_status;
 
 typedef enum { MOBA_BF16 = 0, MOBA_F32 = 1 } moba_dtype;
@@ -259,8 +262,10 @@ MOBA_API moba_status dense_causal_forward(const moba_params* p, const void* q, c
                                  void* stream);
 
 /* Synchronises `stream`, returns the device status word of the current
- * device (MOBA_OK, MOBA_ERR_TIMEOUT or MOBA_ERR_BAD_INDICES) and clears it
- * if `clear` is non-zero. */
+ * device (MOBA_OK, MOBA_ERR_TIMEOUT, MOBA_ERR_BAD_INDICES, MOBA_ERR_INVALID_ARG
+ * for a sequence longer than max_seqlen, or in the checked build
+ * MOBA_ERR_CHECK) and clears it if `clear` is non-zero. The first error
+ * recorded wins. */
 MOBA_API moba_status moba_device_status(void* stream, int clear);
 
 /* Self-test of the bounded waits used by the tensor-core kernels (no paper

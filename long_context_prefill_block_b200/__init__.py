@@ -25,7 +25,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoba.so")
 
 MOBA_OK, MOBA_ERR_INVALID_ARG, MOBA_ERR_UNSUPPORTED, MOBA_ERR_CUDA = 0, -1, -2, -3
-MOBA_ERR_TIMEOUT, MOBA_ERR_WORKSPACE, MOBA_ERR_BAD_INDICES = -4, -5, -6
+MOBA_ERR_TIMEOUT, MOBA_ERR_WORKSPACE, MOBA_ERR_BAD_INDICES, MOBA_ERR_CHECK = -4, -5, -6, -7
 MOBA_BF16, MOBA_F32 = 0, 1
 
 EXPORTS = ("moba_num_blocks", "moba_workspace_size", "moba_meanpool", "moba_gate_topk",

@@ -547,6 +547,7 @@ const char* moba_status_string(moba_status s) {
     case MOBA_ERR_TIMEOUT: return "bounded device wait expired";
     case MOBA_ERR_WORKSPACE: return "workspace missing or too small";
     case MOBA_ERR_BAD_INDICES: return "index row not in canonical form";
+    case MOBA_ERR_CHECK: return "device bounds check failed (checked build)";
   }
   return "unknown status";
 }

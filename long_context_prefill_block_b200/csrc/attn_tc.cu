@@ -244,10 +244,15 @@ template <int MODE>
 __device__ __forceinline__ Row get_row(const Args& a, const Tile& T, int r) {
   const Dims& dm = a.dm;
   Row R{};
+  const int64_t n_part = (int64_t)dm.T * a.ch.nq * dm.topk;  // partial rows of the pass
   if (MODE == HIST) {
-    R.has_q = R.valid = T.row0 + r < T.count;
+    R.has_q = R.valid = T.row0 + r < T.count &&
+                        MOBA_CHECK((int64_t)T.base + T.row0 + r <
+                                       (int64_t)dm.T * a.ch.nq * hist_slots(dm),
+                                   a.status);
     if (R.valid) {
       R.prow = a.pairs[T.base + T.row0 + r];
+      R.has_q = R.valid = MOBA_CHECK(R.prow >= 0 && R.prow < n_part, a.status);
       const int64_t th = R.prow / dm.topk;
       R.t = th / a.ch.nq;
       R.h = a.ch.h0 + (int)(th % a.ch.nq);
@@ -256,7 +261,7 @@ __device__ __forceinline__ Row get_row(const Args& a, const Tile& T, int r) {
   }
   R.h = T.h;
   R.p = T.p0 + r;
-  R.has_q = R.valid = R.p < T.count;
+  R.has_q = R.valid = R.p < T.count && MOBA_CHECK(T.start + R.p < dm.T, a.status);
   R.t = T.start + R.p;
   if (MODE == CUR && R.valid) {
     const int c = R.p / dm.B;
@@ -269,7 +274,8 @@ __device__ __forceinline__ Row get_row(const Args& a, const Tile& T, int r) {
     R.prow = (R.t * a.ch.nq + (R.h - a.ch.h0)) * (int64_t)dm.topk;
     R.own = slot >= 0;
     R.nhist = R.own ? slot : n;
-    R.valid = R.own || dm.prefix;
+    R.valid = (R.own || dm.prefix) &&
+              MOBA_CHECK(R.nhist <= dm.topk && R.prow + dm.topk <= n_part, a.status);
   }
   return R;
 }
@@ -282,12 +288,12 @@ __device__ __forceinline__ bool q_row_of(const Args& a, const Tile& T, int r, in
     const int64_t prow = a.pairs[T.base + T.row0 + r];
     const int64_t th = prow / a.dm.topk;
     qrow = (th / a.ch.nq) * a.dm.Hq + a.ch.h0 + (int)(th % a.ch.nq);
-    return true;
+    return MOBA_CHECK(qrow >= 0 && qrow < (int64_t)a.dm.T * a.dm.Hq, a.status);
   }
   const int p = T.p0 + r;
   if (p >= T.count) return false;
   qrow = (T.start + p) * a.dm.Hq + T.h;
-  return true;
+  return MOBA_CHECK(qrow < (int64_t)a.dm.T * a.dm.Hq, a.status);
 }
 
 __device__ __forceinline__ void regs_dec() {
@@ -767,7 +773,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
         // weight 0.
         const int slot = R.valid ? R.nhist : 0;
         const int64_t prow0 = R.valid ? R.prow : 0;
-        const int64_t orow = R.valid ? R.t * dm.Hq + R.h : -1;
+        const int64_t orow =
+            R.valid && MOBA_CHECK(R.t * dm.Hq + R.h < (int64_t)dm.T * dm.Hq, status)
+                ? R.t * dm.Hq + R.h
+                : -1;
         float o[D];
         {
           // all four loads in flight, then one wait
@@ -788,7 +797,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
         // O[h] is in registers: the next unit's PV may overwrite it
         fence_before_sync();
         mbar_arrive(&sh.o_free[hh]);
-        if (R.valid) {
+        if (orow >= 0) {
           const int64_t nr = (int64_t)a.ch.nq * dm.topk;
           const float m = m_all, L = L_all;
 #pragma unroll
@@ -830,7 +839,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
       } else {
         // Each thread writes its own row in 32-byte pieces (a warp store
         // covers 32 rows; every 32-byte sector is written whole).
-        const int64_t orow = R.valid ? (MODE == DENSE ? R.t * dm.Hq + R.h : R.prow) : -1;
+        const int64_t orow =
+            R.valid && MOBA_CHECK(MODE == DENSE ? R.t * dm.Hq + R.h < (int64_t)dm.T * dm.Hq
+                                                : R.prow < (int64_t)dm.T * a.ch.nq * dm.topk,
+                                  status)
+                ? (MODE == DENSE ? R.t * dm.Hq + R.h : R.prow)
+                : -1;
         const PartRow prt = part_row(R.valid && MODE != DENSE ? R.prow : 0,
                                      (int64_t)a.ch.nq * dm.topk);
         uint32_t ro[D];
@@ -877,7 +891,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ 
             }
           }
         }
-        if (R.valid) {
+        if (orow >= 0) {
           if (MODE == DENSE) {
             if (a.lse_out) a.lse_out[R.t * dm.Hq + R.h] = lse;
           } else {

@@ -15,6 +15,7 @@ constexpr int kF32 = 1;
 constexpr int kStInvalidArg = -1;
 constexpr int kStTimeout = -4;
 constexpr int kStBadIndices = -6;
+constexpr int kStCheck = -7;
 
 // Sizes of one call, validated on the host.
 struct Dims {
@@ -102,6 +103,21 @@ struct Vec16<__nv_bfloat16> {
 __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
+
+// Checked build (MOBA_CHECKED defined: libmoba_checked.so): index and
+// bounds checks at the kernels' computed global accesses. A failed check
+// records kStCheck in the status word and the access is skipped; nothing
+// traps. In the ordinary build MOBA_CHECK(cond, status) is the constant
+// true and costs nothing.
+#ifdef MOBA_CHECKED
+__device__ __forceinline__ bool check_or_flag(bool ok, int* status) {
+  if (!ok) set_status(status, kStCheck);
+  return ok;
+}
+#define MOBA_CHECK(cond, status) (::moba::check_or_flag((cond), (status)))
+#else
+#define MOBA_CHECK(cond, status) (true)
+#endif
 
 // Sequence bounds with a device-side check against max_seqlen.
 __device__ __forceinline__ bool seq_bounds(const Dims& dm, const int32_t* cu, int b, int64_t& start,

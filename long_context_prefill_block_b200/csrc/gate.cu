@@ -213,6 +213,7 @@ __global__ void __launch_bounds__(kThreads) gate_kernel(Dims dm, const T* __rest
     }
   }
   for (int hh = 0; hh < nh; ++hh) {
+    if (!MOBA_CHECK(start + p < dm.T && h0 + hh < dm.Hq, status)) break;
     int32_t* row = idx + ((start + p) * dm.Hq + h0 + hh) * (int64_t)dm.topk;
 #pragma unroll
     for (int r = 0; r <= KM; ++r) {

@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) gate_net_kernel(const NetArgs a) 
           }
           MOBA_TRACE(2, hh);
           const int p = x.p0 + r;
-          const bool has = p < x.len;
+          const bool has = p < x.len && MOBA_CHECK(x.start + p < dm.T && x.h + hh < dm.Hq, status);
           const __nv_bfloat16* src = a.q + ((x.start + (has ? p : 0)) * dm.Hq + x.h + hh) * 128;
           // the row in four 16-column pieces of two 32-byte loads each, one
           // piece's loads in flight while the previous piece is stored (the
@@ -432,6 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) gate_net_kernel(const NetArgs a) 
 #pragma unroll
             for (int u = 0; u < 16; ++u) v[u] = u < hsel ? 255 - (int)sel[u] : (u == hsel ? c : -1);
             for (int hh = 0; hh < nh; ++hh) {
+              if (!MOBA_CHECK(x.start + p < dm.T && x.h + hh < dm.Hq, status)) break;
               int32_t* row = a.idx + ((x.start + p) * dm.Hq + x.h + hh) * (int64_t)dm.topk;
               if (a.vec_rows) {
 #pragma unroll

@@ -387,6 +387,7 @@ gate_tc_kernel(const __grid_constant__ CUtensorMap tmq, const GateArgs a) {
             sel[j + 1] = s;
           }
       for (int hh = 0; hh < nh; ++hh) {
+        if (!MOBA_CHECK(x.start + p < dm.T && x.h + hh < dm.Hq, status)) break;
         int32_t* row = a.idx + ((x.start + p) * dm.Hq + x.h + hh) * (int64_t)dm.topk;
         for (int r = 0; r < dm.topk; ++r)
           row[r] = r < hsel ? sel[r < KM ? r : KM - 1] : (r == hsel && own_in ? c : -1);

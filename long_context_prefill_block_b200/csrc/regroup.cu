@@ -103,7 +103,9 @@ __global__ void __launch_bounds__(kThreads) regroup_pass(Dims dm, Chunk ch,
     if (SCATTER) {
       const int list = list0 + e;
       const int pos = atomicAdd(&cursor[list], 1);
-      pairs[list_off[list] + pos] = (int32_t)(prow0 + slot);
+      const int64_t at = (int64_t)list_off[list] + pos;
+      if (MOBA_CHECK(at < (int64_t)dm.T * ch.nq * hist_slots(dm), status))
+        pairs[at] = (int32_t)(prow0 + slot);
     } else {
       atomicAdd(&counts[list0 + e], 1);
     }
@@ -179,7 +181,9 @@ __global__ void __launch_bounds__(kRows) regroup_pass_smem(Dims dm, Chunk ch,
   if (valid)
     walk_row(row, dm.topk, c, !dm.prefix, [&](int slot, int e) {
       const int pos = base[e] + atomicAdd(&hist[e], 1);
-      pairs[list_off[list0 + e] + pos] = (int32_t)(prow0 + slot);
+      const int64_t at = (int64_t)list_off[list0 + e] + pos;
+      if (MOBA_CHECK(at < (int64_t)dm.T * ch.nq * hist_slots(dm), status))
+        pairs[at] = (int32_t)(prow0 + slot);
     });
 }
 

@@ -36,6 +36,19 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, name), name
 
 
+def test_checked_build_exports_the_same_entry_points():
+    from long_context_prefill_block_b200 import build
+
+    if not os.path.exists(build.LIB_CHECKED):
+        pytest.skip("checked build absent")
+    checked = ctypes.CDLL(build.LIB_CHECKED)
+    for name in declared_symbols():
+        assert hasattr(checked, name), name
+    checked.moba_status_string.argtypes = [ctypes.c_int]
+    checked.moba_status_string.restype = ctypes.c_char_p
+    assert b"check" in checked.moba_status_string(moba.MOBA_ERR_CHECK)
+
+
 def test_trace_entry_points_only_in_the_trace_build():
     from long_context_prefill_block_b200 import build
 
