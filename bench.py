@@ -497,6 +497,7 @@ def bench_decode(args, w, moba, q_all, k, v, cu, dev, world, rank, config, share
     cache (the workload's K/V), through moba_decode; the block means are built once, as a
     serving loop keeps them up to date incrementally."""
     nq_r = args.queries
+    hm = args.kv_layout == "head"
     lens = np.diff(cu.numpy())
     if (lens < nq_r).any():
         raise ValueError("--queries exceeds a sequence length")
@@ -506,8 +507,10 @@ def bench_decode(args, w, moba, q_all, k, v, cu, dev, world, rank, config, share
     del q_all
     cu_d = cu.to(dev)
     cu_q = torch.arange(0, (w.batch + 1) * nq_r, nq_r, dtype=torch.int32)
-    kbar = moba.moba_meanpool(k, cu_d, w.block_size, max_seqlen=w.max_seqlen)
-    p = moba.decode_params(q, k, cu, w.block_size, w.topk, w.max_seqlen, shared)
+    if hm:  # the cache laid out head by head: [Hkv, T, d]
+        k, v = k.transpose(0, 1).contiguous(), v.transpose(0, 1).contiguous()
+    kbar = moba.moba_meanpool(k, cu_d, w.block_size, max_seqlen=w.max_seqlen, kv_head_major=hm)
+    p = moba.decode_params(q, k, cu, w.block_size, w.topk, w.max_seqlen, shared, kv_head_major=hm)
     L = moba.lib()
     L.moba_decode_workspace_size.argtypes = [ctypes.POINTER(moba.MobaParams), ctypes.c_int]
     L.moba_decode_workspace_size.restype = ctypes.c_size_t
@@ -602,7 +605,9 @@ def bench_decode(args, w, moba, q_all, k, v, cu, dev, world, rank, config, share
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
-        "config": dict(config, **{"pass": "decode", "queries_per_request": nq_r}),
+        "config": dict(config, **{"pass": "decode", "queries_per_request": nq_r,
+                                  "kv_layout": "head-major [Hkv, T, d]" if hm else
+                                  "packed [T, Hkv, d]"}),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": None,
                      "kernel": "moba_decode, all launches (gate, split-K attention with the merge)",
@@ -668,6 +673,8 @@ def main():
     ap.add_argument("--pass", dest="pass_", default="forward",
                     choices=["forward", "backward", "decode"])
     ap.add_argument("--queries", type=int, default=1, help="decode: queries per request")
+    ap.add_argument("--kv-layout", default="packed", choices=["packed", "head"],
+                    help="decode: the KV cache packed [T, Hkv, d] or head-major [Hkv, T, d]")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))

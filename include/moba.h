@@ -90,6 +90,13 @@ typedef struct {
                         of it, itself included; its index row then lists only
                         earlier blocks. With routing 1 the group's mean of the
                         own-block scores is used. */
+  int kv_layout;     /* 0 (default): k and v are packed [T][Hkv][d], as everywhere.
+                        1: k and v are head-major [Hkv][T][d] (each kv head's keys
+                        contiguous): a decode KV cache laid out so the split-K
+                        reads of one head stream contiguous rows (section 5.4:
+                        decoding is bound by the KV reads). Accepted by
+                        moba_meanpool, moba_meanpool_update and moba_decode; the
+                        prefill entry points return MOBA_ERR_UNSUPPORTED. */
 } moba_params;
 
 /* Number of key blocks reserved per sequence: ceil(max_seqlen / B). */

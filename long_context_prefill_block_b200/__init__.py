@@ -38,7 +38,8 @@ class MobaParams(ctypes.Structure):
                 ("max_seqlen", ctypes.c_int), ("num_q_heads", ctypes.c_int),
                 ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
                 ("block_size", ctypes.c_int), ("topk", ctypes.c_int), ("dtype", ctypes.c_int),
-                ("routing", ctypes.c_int), ("own_block", ctypes.c_int)]
+                ("routing", ctypes.c_int), ("own_block", ctypes.c_int),
+                ("kv_layout", ctypes.c_int)]
 
 
 class MobaError(RuntimeError):
@@ -179,14 +180,26 @@ def workspace(params: MobaParams, device) -> torch.Tensor:
     return torch.empty(max(moba_workspace_size(params), 256), dtype=torch.uint8, device=device)
 
 
+def _packed_view(k: torch.Tensor, head_major: bool) -> torch.Tensor:
+    """The [T, Hkv, d] shape of a cache given [Hkv, T, d] when head_major (shape checks only)."""
+    if not head_major:
+        return k
+    if k.dim() != 3:
+        raise ValueError("a head-major cache must be [Hkv, T, d]")
+    return k.transpose(0, 1)
+
+
 def moba_meanpool(k: torch.Tensor, cu_seqlens: torch.Tensor, block_size: int,
-                  max_seqlen: Optional[int] = None) -> torch.Tensor:
-    """Block means fp32 [batch, num_blocks, Hkv, d]."""
-    _check_qkv(k, k)
-    _check_cu(cu_seqlens, k.shape[0])
+                  max_seqlen: Optional[int] = None, kv_head_major: bool = False) -> torch.Tensor:
+    """Block means fp32 [batch, num_blocks, Hkv, d]. k: [T, Hkv, d], or [Hkv, T, d] with
+    kv_head_major (a decode cache laid out head by head)."""
+    kp = _packed_view(k, kv_head_major)
+    _check_qkv(kp, kp)
+    _check_cu(cu_seqlens, kp.shape[0])
     _check_inputs(k)
-    p = make_params(k, k, cu_seqlens, block_size, 1, max_seqlen)
+    p = make_params(kp, kp, cu_seqlens, block_size, 1, max_seqlen)
     p.num_q_heads = p.num_kv_heads
+    p.kv_layout = 1 if kv_head_major else 0
     cu = _dev_i32(cu_seqlens, k.device)
     kbar = torch.empty((p.batch, moba_num_blocks(p), p.num_kv_heads, p.head_dim),
                        dtype=torch.float32, device=k.device)
@@ -197,14 +210,17 @@ def moba_meanpool(k: torch.Tensor, cu_seqlens: torch.Tensor, block_size: int,
 
 def moba_meanpool_update(k_cache: torch.Tensor, cu_seqlens: torch.Tensor, cu_new: torch.Tensor,
                          kbar: torch.Tensor, block_size: int, max_new: int,
-                         max_seqlen: Optional[int] = None) -> torch.Tensor:
+                         max_seqlen: Optional[int] = None,
+                         kv_head_major: bool = False) -> torch.Tensor:
     """Recompute, in place, the block means kbar [batch, num_blocks, Hkv, d] of the blocks that
     hold each request's last cu_new[r+1] - cu_new[r] cache positions (just appended)."""
-    _check_qkv(k_cache, k_cache)
-    _check_cu(cu_seqlens, k_cache.shape[0])
+    kp = _packed_view(k_cache, kv_head_major)
+    _check_qkv(kp, kp)
+    _check_cu(cu_seqlens, kp.shape[0])
     _check_inputs(k_cache, kbar)
-    p = make_params(k_cache, k_cache, cu_seqlens, block_size, 1, max_seqlen)
+    p = make_params(kp, kp, cu_seqlens, block_size, 1, max_seqlen)
     p.num_q_heads = p.num_kv_heads
+    p.kv_layout = 1 if kv_head_major else 0
     cu = _dev_i32(cu_seqlens, k_cache.device)
     cn = _dev_i32(cu_new, k_cache.device)
     fn = lib().moba_meanpool_update
@@ -218,27 +234,32 @@ def moba_meanpool_update(k_cache: torch.Tensor, cu_seqlens: torch.Tensor, cu_new
 
 
 def decode_params(q, k_cache, cu_seqlens, block_size: int, topk: int, max_seqlen=None,
-                  shared_routing: bool = False) -> MobaParams:
+                  shared_routing: bool = False, kv_head_major: bool = False) -> MobaParams:
     """Parameters of a decode step: the cache's shape with q's heads."""
-    p = make_params(k_cache, k_cache, cu_seqlens, block_size, topk, max_seqlen, shared_routing)
+    kp = _packed_view(k_cache, kv_head_major)
+    p = make_params(kp, kp, cu_seqlens, block_size, topk, max_seqlen, shared_routing)
     p.num_q_heads = q.shape[1]
+    p.kv_layout = 1 if kv_head_major else 0
     return p
 
 
 def moba_decode(q, k_cache, v_cache, cu_seqlens, cu_q, kbar, block_size: int, topk: int,
                 max_seqlen=None, shared_routing: bool = False, return_lse: bool = False,
                 return_idx: bool = False, ws: Optional[torch.Tensor] = None,
-                out: Optional[torch.Tensor] = None):
+                out: Optional[torch.Tensor] = None, kv_head_major: bool = False):
     """Decode step: request r's queries (rows cu_q[r] .. cu_q[r+1]-1 of q [n, Hq, d]) sit at the
-    last positions of its cache (tokens cu_seqlens[r] .. cu_seqlens[r+1]-1 of k_cache, v_cache);
-    kbar: the cache's block means. Returns out [n, Hq, d] (and lse [n, Hq], idx [n, Hq, topk])."""
-    _check_qkv(k_cache, k_cache, v_cache)
+    last positions of its cache (tokens cu_seqlens[r] .. cu_seqlens[r+1]-1 of k_cache, v_cache:
+    [T, Hkv, d], or [Hkv, T, d] with kv_head_major); kbar: the cache's block means. Returns
+    out [n, Hq, d] (and lse [n, Hq], idx [n, Hq, topk])."""
+    kp, vp = _packed_view(k_cache, kv_head_major), _packed_view(v_cache, kv_head_major)
+    _check_qkv(kp, kp, vp)
     if q.dim() != 3 or q.dtype != k_cache.dtype or q.shape[2] != k_cache.shape[2]:
         raise ValueError("q must be [n, Hq, d] in the cache's dtype and head dim")
-    _check_cu(cu_seqlens, k_cache.shape[0])
+    _check_cu(cu_seqlens, kp.shape[0])
     _check_inputs(q, k_cache, v_cache, kbar, out)
     L = lib()
-    p = decode_params(q, k_cache, cu_seqlens, block_size, topk, max_seqlen, shared_routing)
+    p = decode_params(q, k_cache, cu_seqlens, block_size, topk, max_seqlen, shared_routing,
+                      kv_head_major)
     n = q.shape[0]
     cu = _dev_i32(cu_seqlens, q.device)
     cq = _dev_i32(cu_q, q.device)

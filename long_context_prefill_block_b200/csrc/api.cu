@@ -41,6 +41,7 @@ moba_status validate(const moba_params* p, Dims& dm) {
     return MOBA_ERR_INVALID_ARG;
   if (p->routing != 0 && p->routing != 1) return MOBA_ERR_INVALID_ARG;
   if (p->own_block != 0 && p->own_block != 1) return MOBA_ERR_INVALID_ARG;
+  if (p->kv_layout != 0 && p->kv_layout != 1) return MOBA_ERR_INVALID_ARG;
   if (p->dtype != MOBA_BF16 && p->dtype != MOBA_F32) return MOBA_ERR_UNSUPPORTED;
   if (p->head_dim != 64 && p->head_dim != 128) return MOBA_ERR_UNSUPPORTED;
   if (p->topk > 32) return MOBA_ERR_UNSUPPORTED;
@@ -59,6 +60,7 @@ moba_status validate(const moba_params* p, Dims& dm) {
   dm.dtype = p->dtype == MOBA_BF16 ? kBF16 : kF32;
   dm.shared = p->routing;
   dm.prefix = p->own_block;
+  dm.kv_hm = p->kv_layout;
   return MOBA_OK;
 }
 
@@ -168,6 +170,7 @@ moba_status forward_impl(const moba_params* p, const void* q, const void* k, con
   Dims dm;
   moba_status s = validate(p, dm);
   if (s != MOBA_OK) return s;
+  if (dm.kv_hm) return MOBA_ERR_UNSUPPORTED;  // head-major k / v: decode caches only
   if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
   if (!q || !k || !v || !cu || !out) return MOBA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
@@ -281,6 +284,7 @@ moba_status backward_impl(const moba_params* p, const void* q, const void* k, co
   Dims dm;
   moba_status s = validate(p, dm);
   if (s != MOBA_OK) return s;
+  if (dm.kv_hm) return MOBA_ERR_UNSUPPORTED;
   if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
   if (!q || !k || !v || !cu || !out || !lse || !dout || !dq || !dk || !dv)
     return MOBA_ERR_INVALID_ARG;
@@ -452,6 +456,7 @@ moba_status moba_gate_topk(const moba_params* p, const void* q, const void* k,
   Dims dm;
   moba_status s = validate(p, dm);
   if (s != MOBA_OK) return s;
+  if (dm.kv_hm) return MOBA_ERR_UNSUPPORTED;
   if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
   if (!q || !k || !cu_seqlens || !idx || !aligned16(q) || !aligned16(k)) return MOBA_ERR_INVALID_ARG;
   // the gate needs the block means and, for the prefix-mean variant, the
@@ -507,6 +512,7 @@ moba_status dense_causal_forward(const moba_params* p, const void* q, const void
   Dims dm;
   moba_status s = validate(p, dm);
   if (s != MOBA_OK) return s;
+  if (dm.kv_hm) return MOBA_ERR_UNSUPPORTED;
   if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
   if (!q || !k || !v || !cu_seqlens || !out) return MOBA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||

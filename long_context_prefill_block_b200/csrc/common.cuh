@@ -30,7 +30,13 @@ struct Dims {
   int dtype;       // kBF16 / kF32
   int shared;      // 1: a kv head's query heads share the blocks of their mean score
   int prefix;      // 1: the own block is scored by its prefix mean instead of forced
+  int kv_hm;       // 1: k and v are head-major [Hkv][T][d] (decode caches), else [T][Hkv][d]
 };
+
+// Element offset of row t of kv head g in k or v.
+__host__ __device__ __forceinline__ int64_t kv_row(const Dims& dm, int64_t t, int g) {
+  return (dm.kv_hm ? (int64_t)g * dm.T + t : t * dm.Hkv + g) * dm.d;
+}
 
 // History slots an index row can hold: k - 1 beside the forced own block,
 // all k when the own block competes for its slot.

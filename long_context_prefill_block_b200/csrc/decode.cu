@@ -262,9 +262,11 @@ decode_attn_kernel(Dims dm, const T* __restrict__ q, const T* __restrict__ k,
   float m = -INFINITY, l = 0.f, o[EPL];
 #pragma unroll
   for (int x = 0; x < EPL; ++x) o[x] = 0.f;
-  const T* kbase = k + (start * dm.Hkv + g) * (int64_t)D + sub * EPL;
-  const T* vbase = v + (start * dm.Hkv + g) * (int64_t)D + sub * EPL;
-  const int64_t rs = (int64_t)dm.Hkv * D;  // row stride of the cache
+  const T* kbase = k + kv_row(dm, start, g) + sub * EPL;
+  const T* vbase = v + kv_row(dm, start, g) + sub * EPL;
+  // row stride of the cache: a head-major cache keeps one head's rows
+  // contiguous, so a split streams consecutive rows
+  const int64_t rs = dm.kv_hm ? (int64_t)D : (int64_t)dm.Hkv * D;
   // The trip count is the same for every lane (the shuffles need all 32).
   // A step loads U rows per lane group as raw 16-byte vectors (all 2U loads
   // in flight together), then folds them into the softmax with one rescale.

@@ -67,8 +67,9 @@ extern "C" moba_status moba_gate_topk_noalloc(const moba_params* p, const void* 
   moba::Dims dm;
   const moba_status s = moba::validate(p, dm);
   if (s != MOBA_OK) return s;
-  // the prefix-mean gate keeps T * Hq own-block scores: no room in the fixed array
-  if (dm.prefix) return MOBA_ERR_UNSUPPORTED;
+  // the prefix-mean gate keeps T * Hq own-block scores: no room in the fixed
+  // array; head-major k is a decode-cache layout, which no gate call takes
+  if (dm.prefix || dm.kv_hm) return MOBA_ERR_UNSUPPORTED;
   if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
   // the size limit is checked before the pointers, so that a refusal never
   // depends on what the pointers hold

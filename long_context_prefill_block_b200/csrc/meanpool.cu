@@ -1,6 +1,7 @@
 // Block mean-pooling of keys (PaperTrace "2.1.3 MoBA", section 1, eq. 3):
 // kbar_i = (1/B) * sum of the raw keys of block i, one routing vector per
-// (sequence, block, kv head), fp32.
+// (sequence, block, kv head), fp32. Keys packed [T][Hkv][d] or, for decode
+// caches, head-major [Hkv][T][d].
 //
 // One CTA per (block, sequence, kv head). Each thread owns 16 bytes of a key
 // row (8 bf16 or 4 fp32 elements); a row is read by D*size/16 consecutive
@@ -57,7 +58,7 @@ __global__ void __launch_bounds__(kThreads) meanpool_kernel(Dims dm, const T* __
 #pragma unroll 8
   for (int j = j0 + rg; j < j1; j += RG) {
     float x[VEC];
-    Vec16<T>::load(k + ((start + j) * dm.Hkv + g) * (int64_t)D + lane * VEC, x);
+    Vec16<T>::load(k + kv_row(dm, start + j, g) + lane * VEC, x);
 #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] += x[e];
   }

@@ -150,3 +150,56 @@ def test_decode_at_scaling_size():
     assert moba.moba_device_status() == 0
     _check(q_all.cpu(), k.cpu(), v.cpu(), cu, w.block_size, w.topk, rows, out.cpu(), lse.cpu(),
            idx.cpu())
+
+
+@pytest.mark.parametrize("case", CASES[:4])
+def test_decode_head_major_cache(case):
+    # the same caches laid out head by head ([Hkv, T, d], moba_params.kv_layout = 1): the
+    # block means and the decode results are bit-identical to the packed cache's, and the
+    # oracle agrees; an append refreshes the means in the head-major layout too
+    lengths, Hq, Hkv, d, B, topk, dtype, n_new = case
+    q_all, k, v, cu = small_case(lengths, Hq, Hkv, d, B, topk, dtype=dtype, seed=441)
+    rows, out, lse, idx = _run_decode(q_all, k, v, cu, n_new, B, topk)
+    tok = torch.as_tensor(rows[::Hq] // Hq)
+    q = q_all[tok].contiguous().to(DEV)
+    cu_q = torch.tensor(np.concatenate([[0], np.cumsum(n_new)]), dtype=torch.int32)
+    kh = k.transpose(0, 1).contiguous().to(DEV)
+    vh = v.transpose(0, 1).contiguous().to(DEV)
+    kbar_p = moba.moba_meanpool(k.to(DEV), cu.to(DEV), B)
+    kbar_h = moba.moba_meanpool(kh, cu.to(DEV), B, kv_head_major=True)
+    out_h, lse_h, idx_h = moba.moba_decode(q, kh, vh, cu, cu_q, kbar_h, B, topk, return_lse=True,
+                                           return_idx=True, kv_head_major=True)
+    torch.cuda.synchronize()
+    assert moba.moba_device_status() == 0
+    assert torch.equal(kbar_h, kbar_p)
+    assert torch.equal(idx_h.cpu(), idx) and torch.equal(lse_h.cpu(), lse)
+    assert torch.equal(out_h.cpu(), out)
+    _check(q_all, k, v, cu, B, topk, rows, out_h.cpu(), lse_h.cpu(), idx_h.cpu())
+    # incremental block means: recompute the blocks of each request's last positions
+    kbar_u = kbar_h.clone()
+    kbar_u[:] = 0
+    cu_new = torch.tensor(np.concatenate([[0], np.cumsum(n_new)]), dtype=torch.int32)
+    moba.moba_meanpool_update(kh, cu.to(DEV), cu_new, kbar_u, B, max(max(n_new), 1),
+                              kv_head_major=True)
+    torch.cuda.synchronize()
+    for r, n in enumerate(n_new):
+        L = int(cu[r + 1] - cu[r])
+        for blk in sorted({(L - 1 - j) // B for j in range(n)}):
+            assert torch.equal(kbar_u[r, blk], kbar_p[r, blk])
+
+
+def test_prefill_refuses_head_major_kv():
+    q, k, v, cu = small_case((300,), 2, 2, 128, 128, 3, dtype=torch.bfloat16, seed=442)
+    p = moba.make_params(q, k, cu, 128, 3)
+    p.kv_layout = 1
+    ws = moba.workspace(p, DEV)
+    L = moba.lib()
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    out = torch.empty_like(qd)
+    cu_d = cu.to(DEV)
+    ptr = lambda x: moba.ctypes.c_void_p(x.data_ptr())
+    rc = L.moba_forward(moba.ctypes.byref(p), ptr(qd), ptr(kd), ptr(vd), ptr(cu_d), ptr(out), None,
+                        ptr(ws), ws.numel(), None)
+    assert rc == moba.MOBA_ERR_UNSUPPORTED
+    p.kv_layout = 2
+    assert moba.moba_workspace_size(p) == 0  # invalid layout value
