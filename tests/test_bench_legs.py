@@ -106,3 +106,17 @@ def test_reference_arm_prints_one_line():
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["config"]["workload"] == "tiny_fp32"
+
+
+def test_run_cli_workload_overrides():
+    """The profiling CLI keeps the named workload's heads, dtype and seed and only replaces
+    the shape fields it is given (one sequence of --tokens)."""
+    from long_context_prefill_block_b200.run import workload
+    from moba_inputs import WORKLOADS
+    base = WORKLOADS["llama_1m"]
+    assert workload("llama_1m", None, None, None) is base
+    w = workload("llama_1m", 131072, 512, None)
+    assert w.lengths == (131072,) and w.block_size == 512 and w.topk == base.topk
+    assert (w.num_q_heads, w.num_kv_heads, w.head_dim, w.dtype, w.seed) == \
+        (base.num_q_heads, base.num_kv_heads, base.head_dim, base.dtype, base.seed)
+    assert -(-w.max_seqlen // w.block_size) == 256  # the million-token gate's block count
