@@ -23,9 +23,11 @@
  * Element type: bf16 or fp32 (moba_params.dtype) for q, k, v and out;
  *   arithmetic is fp32 (bf16 tensor-core products, fp32 accumulation).
  * Pointers: every data pointer is a DEVICE pointer owned by the caller,
- *   16-byte aligned. cu_seqlens is a device pointer too. The library never
- *   allocates device memory, never frees, and never synchronises the stream;
- *   temporary storage comes from the caller's workspace.
+ *   32-byte aligned (the kernels move rows in 32-byte pieces; every PyTorch
+ *   allocation and any view of whole rows qualifies), and so is a workspace.
+ *   cu_seqlens is a device pointer too. The library never allocates device
+ *   memory, never frees, and never synchronises the stream; temporary
+ *   storage comes from the caller's workspace.
  * Stream: `stream` is a cudaStream_t passed as void* (NULL = legacy default).
  * Errors: arguments are validated on the host before anything is launched;
  *   an invalid call returns a negative moba_status and launches nothing.
@@ -209,7 +211,7 @@ MOBA_API moba_status moba_forward_with_indices(const moba_params* p, const void*
  *   idx: the forward's index rows [T][Hq][k] (canonical form), or NULL to
  *   run the gate again (p->routing as in the forward).
  *   dq [T][Hq][d], dk and dv [T][Hkv][d]: fp32, caller-owned, overwritten.
- *   ws: moba_backward_workspace_size(p, idx != NULL) bytes, 16-byte aligned.
+ *   ws: moba_backward_workspace_size(p, idx != NULL) bytes, 32-byte aligned.
  * Errors as moba_forward (MOBA_ERR_BAD_INDICES via the status word). */
 MOBA_API size_t moba_backward_workspace_size(const moba_params* p, int have_indices);
 MOBA_API moba_status moba_backward(const moba_params* p, const void* q, const void* k,
@@ -242,7 +244,7 @@ MOBA_API moba_status moba_backward(const moba_params* p, const void* q, const vo
  *   out: [n_queries][Hq][d] (p->dtype); lse: fp32 [n_queries][Hq] or NULL;
  *   idx: int32 [n_queries][Hq][k] receives the chosen blocks (canonical
  *      form), or NULL.
- *   ws: moba_decode_workspace_size(p, n_queries) bytes, 16-byte aligned. */
+ *   ws: moba_decode_workspace_size(p, n_queries) bytes, 32-byte aligned. */
 MOBA_API size_t moba_decode_workspace_size(const moba_params* p, int n_queries);
 MOBA_API moba_status moba_decode(const moba_params* p, const void* q, const void* k_cache,
                                  const void* v_cache, const int32_t* cu_seqlens,

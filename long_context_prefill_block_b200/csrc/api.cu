@@ -82,7 +82,7 @@ constexpr size_t kPartialCap = size_t(32) << 30;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; }
+bool aligned32(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 31) == 0; }
 
 struct Layout {
   size_t kbar, own, idx, counts, cursor, list_off, tile_off, pairs, tiles, part_o, part_lse, total;
@@ -173,11 +173,11 @@ moba_status forward_impl(const moba_params* p, const void* q, const void* k, con
   if (dm.kv_hm) return MOBA_ERR_UNSUPPORTED;  // head-major k / v: decode caches only
   if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
   if (!q || !k || !v || !cu || !out) return MOBA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-      (lse && !aligned16(lse)))
+  if (!aligned32(q) || !aligned32(k) || !aligned32(v) || !aligned32(out) ||
+      (lse && !aligned32(lse)))
     return MOBA_ERR_INVALID_ARG;
   const Layout L = plan(dm, idx_in == nullptr);
-  if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOBA_ERR_WORKSPACE;
+  if (!ws || ws_bytes < L.total || !aligned32(ws)) return MOBA_ERR_WORKSPACE;
   if (events && n_events < 3 + 4 * num_passes(dm, L)) return MOBA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int ev = 0;
@@ -290,9 +290,9 @@ moba_status backward_impl(const moba_params* p, const void* q, const void* k, co
     return MOBA_ERR_INVALID_ARG;
   for (const void* x : {q, k, v, out, dout, static_cast<const void*>(dq),
                         static_cast<const void*>(dk), static_cast<const void*>(dv)})
-    if (!aligned16(x)) return MOBA_ERR_INVALID_ARG;
+    if (!aligned32(x)) return MOBA_ERR_INVALID_ARG;
   const BwdLayout L = plan_bwd(dm, idx_in == nullptr);
-  if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOBA_ERR_WORKSPACE;
+  if (!ws || ws_bytes < L.total || !aligned32(ws)) return MOBA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int* status = status_word();
   if (!status) return MOBA_ERR_CUDA;
@@ -379,11 +379,11 @@ moba_status moba_decode(const moba_params* p, const void* q, const void* k_cache
   if ((int64_t)n_queries * dm.Hq * dm.topk >= (int64_t(1) << 31)) return MOBA_ERR_UNSUPPORTED;
   if (!q || !k_cache || !v_cache || !cu_seqlens || !cu_q || !kbar || !out)
     return MOBA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(kbar) ||
-      !aligned16(out))
+  if (!aligned32(q) || !aligned32(k_cache) || !aligned32(v_cache) || !aligned32(kbar) ||
+      !aligned32(out))
     return MOBA_ERR_INVALID_ARG;
   const DecLayout L = plan_decode(dm, n_queries);
-  if (!ws || ws_bytes < L.total || !aligned16(ws)) return MOBA_ERR_WORKSPACE;
+  if (!ws || ws_bytes < L.total || !aligned32(ws)) return MOBA_ERR_WORKSPACE;
   int* status = status_word();
   if (!status) return MOBA_ERR_CUDA;
   char* base = static_cast<char*>(ws);
@@ -403,7 +403,7 @@ moba_status moba_meanpool_update(const moba_params* p, const void* k_cache,
   if (s != MOBA_OK) return s;
   if (max_new < 0) return MOBA_ERR_INVALID_ARG;
   if (dm.batch == 0 || dm.nb == 0 || max_new == 0) return MOBA_OK;
-  if (!k_cache || !cu_seqlens || !cu_new || !kbar || !aligned16(k_cache) || !aligned16(kbar))
+  if (!k_cache || !cu_seqlens || !cu_new || !kbar || !aligned32(k_cache) || !aligned32(kbar))
     return MOBA_ERR_INVALID_ARG;
   int* status = status_word();
   if (!status) return MOBA_ERR_CUDA;
@@ -443,7 +443,7 @@ moba_status moba_meanpool(const moba_params* p, const void* k, const int32_t* cu
   moba_status s = validate(p, dm);
   if (s != MOBA_OK) return s;
   if (dm.batch == 0 || dm.nb == 0) return MOBA_OK;
-  if (!k || !cu_seqlens || !kbar || !aligned16(k) || !aligned16(kbar)) return MOBA_ERR_INVALID_ARG;
+  if (!k || !cu_seqlens || !kbar || !aligned32(k) || !aligned32(kbar)) return MOBA_ERR_INVALID_ARG;
   int* status = status_word();
   if (!status) return MOBA_ERR_CUDA;
   return cuda_status(launch_meanpool(dm, k, cu_seqlens, kbar, status,
@@ -458,13 +458,13 @@ moba_status moba_gate_topk(const moba_params* p, const void* q, const void* k,
   if (s != MOBA_OK) return s;
   if (dm.kv_hm) return MOBA_ERR_UNSUPPORTED;
   if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
-  if (!q || !k || !cu_seqlens || !idx || !aligned16(q) || !aligned16(k)) return MOBA_ERR_INVALID_ARG;
+  if (!q || !k || !cu_seqlens || !idx || !aligned32(q) || !aligned32(k)) return MOBA_ERR_INVALID_ARG;
   // the gate needs the block means and, for the prefix-mean variant, the
   // own-block scores: the head of the forward's workspace plan
   const Layout L = plan(dm, true);
   const size_t need = dm.prefix ? L.own + own_score_bytes(dm, true)
                                 : L.kbar + sizeof(float) * (size_t)dm.batch * dm.nb * dm.Hkv * dm.d;
-  if (!ws || ws_bytes < need || !aligned16(ws)) return MOBA_ERR_WORKSPACE;
+  if (!ws || ws_bytes < need || !aligned32(ws)) return MOBA_ERR_WORKSPACE;
   int* status = status_word();
   if (!status) return MOBA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -515,8 +515,8 @@ moba_status dense_causal_forward(const moba_params* p, const void* q, const void
   if (dm.kv_hm) return MOBA_ERR_UNSUPPORTED;
   if (dm.T == 0 || dm.batch == 0) return MOBA_OK;
   if (!q || !k || !v || !cu_seqlens || !out) return MOBA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-      (lse && !aligned16(lse)))
+  if (!aligned32(q) || !aligned32(k) || !aligned32(v) || !aligned32(out) ||
+      (lse && !aligned32(lse)))
     return MOBA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int* status = status_word();

@@ -57,7 +57,7 @@ cudaError_t addresses_on_current_device(float** scratch, int** status) {
   return cudaSuccess;
 }
 
-bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; }
+bool aligned32(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 31) == 0; }
 
 }  // namespace
 
@@ -75,7 +75,7 @@ extern "C" moba_status moba_gate_topk_noalloc(const moba_params* p, const void* 
   // depends on what the pointers hold
   const size_t need = sizeof(float) * (size_t)dm.batch * dm.nb * dm.Hkv * dm.d;
   if (need > kScratchBytes) return MOBA_ERR_WORKSPACE;  // beyond the built-in 4 MiB
-  if (!q || !k || !cu_seqlens || !idx || !aligned16(q) || !aligned16(k))
+  if (!q || !k || !cu_seqlens || !idx || !aligned32(q) || !aligned32(k))
     return MOBA_ERR_INVALID_ARG;
   float* kbar = nullptr;
   int* status = nullptr;

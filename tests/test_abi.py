@@ -122,6 +122,14 @@ def test_null_and_misaligned_pointers_rejected_before_launch():
     # workspace too small
     assert lib.moba_forward(ctypes.byref(p), fake, fake, fake, fake, fake, None, fake, 16,
                             None) == moba.MOBA_ERR_WORKSPACE
+    # 16-byte but not 32-byte aligned: the kernels move rows in 32-byte pieces
+    half = ctypes.c_void_p((1 << 20) + 16)
+    assert lib.moba_forward(ctypes.byref(p), half, fake, fake, fake, fake, None, fake, 1 << 40,
+                            None) == moba.MOBA_ERR_INVALID_ARG
+    assert lib.moba_forward(ctypes.byref(p), fake, fake, fake, fake, half, None, fake, 1 << 40,
+                            None) == moba.MOBA_ERR_INVALID_ARG
+    assert lib.moba_forward(ctypes.byref(p), fake, fake, fake, fake, fake, None, half, 1 << 40,
+                            None) == moba.MOBA_ERR_WORKSPACE
     assert lib.dense_causal_forward(ctypes.byref(p), fake, None, fake, fake, fake, None,
                                     None) == moba.MOBA_ERR_INVALID_ARG
 
