@@ -62,6 +62,7 @@ sys.path.insert(0, ROOT)
 from moba_inputs import WORKLOADS, make_inputs, sample_rows  # noqa: E402
 
 METRIC = "moba_prefill_fwd_useful_tflops"
+SIDE_WORKLOADS = ("long_32k", "micro_32k")
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 DEFAULT_WORKLOAD = "llama_1m"
 TIE_GAP = 1e-4  # near-tie band of the block indices (relative score gap)
@@ -625,6 +626,95 @@ def bench_decode(args, w, moba, q_all, k, v, cu, dev, world, rank, config, share
         torch.distributed.destroy_process_group()
 
 
+def stage_times(L, P, bufs, stream, dev, reps: int):
+    """Per-stage milliseconds of moba_forward_staged: CUDA events the library
+    records on the launching stream between its stages, mean of `reps` calls."""
+    q, k, v, cu_d, out, ws = bufs
+    vp = lambda x: ctypes.c_void_p(x.data_ptr())
+    n_pass = L.moba_num_passes(P)
+    n_ev = 3 + 4 * n_pass
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    for e in evs:  # torch creates the CUDA event on first record
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    ev_arr = (ctypes.c_void_p * n_ev)(*[ctypes.c_void_p(e.cuda_event) for e in evs])
+    stage_ms = {"meanpool": 0.0, "gate_topk": 0.0, "regroup": 0.0, "attn_history": 0.0,
+                "attn_current": 0.0, "merge": 0.0}
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    for _ in range(reps):
+        rc = L.moba_forward_staged(P, vp(q), vp(k), vp(v), vp(cu_d), vp(out), None, vp(ws),
+                                   ws.numel(), ev_arr, n_ev, sp)
+        if rc:
+            raise RuntimeError(f"moba_forward_staged failed: {rc}")
+        torch.cuda.synchronize(dev)
+        stage_ms["meanpool"] += evs[0].elapsed_time(evs[1]) / reps
+        stage_ms["gate_topk"] += evs[1].elapsed_time(evs[2]) / reps
+        prev = evs[2]
+        for j in range(n_pass):
+            a, b_, c_, d_ = evs[3 + 4 * j: 7 + 4 * j]
+            stage_ms["regroup"] += prev.elapsed_time(a) / reps
+            stage_ms["attn_history"] += a.elapsed_time(b_) / reps
+            stage_ms["attn_current"] += b_.elapsed_time(c_) / reps
+            stage_ms["merge"] += c_.elapsed_time(d_) / reps
+            prev = d_
+    return stage_ms
+
+
+def side_workload(name: str, moba, dev, burst: float):
+    """The forward at another workload, timed like the headline one (CUDA events,
+    3 warm-up steps, about a second of timed steps; inputs larger than L2), with
+    its attention-kernel fraction of the burst peak and the dense causal time, so
+    that the 32K shapes sit beside the million-token line in one run."""
+    w = WORKLOADS[name]
+    q, k, v, cu = make_inputs(w, dev)
+    cu_d = cu.to(dev)
+    p = moba.make_params(q, k, cu, w.block_size, w.topk, w.max_seqlen)
+    ws = moba.workspace(p, dev)
+    out = torch.empty_like(q)
+    L, P = moba.lib(), ctypes.byref(p)
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    vp = lambda x: ctypes.c_void_p(x.data_ptr())
+
+    def step():
+        rc = L.moba_forward(P, vp(q), vp(k), vp(v), vp(cu_d), vp(out), None, vp(ws), ws.numel(),
+                            sp)
+        if rc:
+            raise RuntimeError(f"moba_forward failed: {rc}")
+
+    t_w = time.perf_counter()
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    warm_s = (time.perf_counter() - t_w) / 3
+    steps = int(min(200, max(5, round(1.0 / max(warm_s, 1e-4)))))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if moba.moba_device_status(dev) != 0:
+        raise RuntimeError(f"device status error at {name}")
+    ms = e0.elapsed_time(e1) / steps
+    useful, hist_flops, _, _ = flop_counts(w)
+    st = stage_times(L, P, (q, k, v, cu_d, out, ws), stream, dev, 5)
+    attn_ms = st["attn_history"] + st["attn_current"] + st["merge"]
+    dense = torch.empty_like(q)
+    moba.dense_causal_forward(q, k, v, cu, max_seqlen=w.max_seqlen, out=dense)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for _ in range(3):
+        moba.dense_causal_forward(q, k, v, cu, max_seqlen=w.max_seqlen, out=dense)
+    d1.record(stream)
+    torch.cuda.synchronize(dev)
+    dense_ms = d0.elapsed_time(d1) / 3
+    return {"ms_per_step": ms, "steps": steps, "useful_tflops": useful / (ms * 1e-3) / 1e12,
+            "attn_kernels_frac_of_burst": useful / (attn_ms * 1e-3) / 1e12 / burst,
+            "history_frac_of_burst": hist_flops / (st["attn_history"] * 1e-3) / 1e12 / burst,
+            "stage_ms": st, "dense_causal_ms": dense_ms, "speedup_vs_dense": dense_ms / ms}
+
+
 def run_reference(args, w, config):
     """--impl reference: the fp64 oracle on the host cores, each step a
     bounded seeded row sample of the workload, same input bits as the GPU arm."""
@@ -669,6 +759,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-hash", action="store_true", help="skip the input SHA-256s")
+    ap.add_argument("--no-side", action="store_true",
+                    help="skip the forward at the 32K shapes beside the headline workload")
     ap.add_argument("--variant", default="forced", choices=["forced", "shared", "prefix"])
     ap.add_argument("--pass", dest="pass_", default="forward",
                     choices=["forward", "backward", "decode"])
@@ -786,31 +878,8 @@ def main():
 
     # ---- per-stage timing (same stream, CUDA events recorded by the library)
     n_pass = L.moba_num_passes(P)
-    n_ev = 3 + 4 * n_pass
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-    for e in evs:  # torch creates the CUDA event on first record
-        e.record(stream)
-    torch.cuda.synchronize(dev)
-    ev_arr = (ctypes.c_void_p * n_ev)(*[ctypes.c_void_p(e.cuda_event) for e in evs])
-    stage_ms = {"meanpool": 0.0, "gate_topk": 0.0, "regroup": 0.0, "attn_history": 0.0,
-                "attn_current": 0.0, "merge": 0.0}
     reps = 3 if long_step else max(3, min(args.steps, 10))
-    for _ in range(reps):
-        rc = L.moba_forward_staged(P, vp(q), vp(k), vp(v), vp(cu_d), vp(out), None, vp(ws),
-                                   ws.numel(), ev_arr, n_ev, sp)
-        if rc:
-            raise RuntimeError(f"moba_forward_staged failed: {rc}")
-        torch.cuda.synchronize(dev)
-        stage_ms["meanpool"] += evs[0].elapsed_time(evs[1]) / reps
-        stage_ms["gate_topk"] += evs[1].elapsed_time(evs[2]) / reps
-        prev = evs[2]
-        for j in range(n_pass):
-            a, b_, c_, d_ = evs[3 + 4 * j: 7 + 4 * j]
-            stage_ms["regroup"] += prev.elapsed_time(a) / reps
-            stage_ms["attn_history"] += a.elapsed_time(b_) / reps
-            stage_ms["attn_current"] += b_.elapsed_time(c_) / reps
-            stage_ms["merge"] += c_.elapsed_time(d_) / reps
-            prev = d_
+    stage_ms = stage_times(L, P, (q, k, v, cu_d, out, ws), stream, dev, reps)
 
     # ---- dense causal comparison at the same shape
     # (seconds-long dense passes, as at the million-token shape: one warm-up, one timed)
@@ -929,6 +998,10 @@ def main():
         del out_c, lse_c, idx_c
         parity = parity_stats(w, leg, hk, hv, cu, got_out, got_lse, got_idx)
     hashes = None if args.no_hash else input_hashes({"q": hq, "k": hk, "v": hv, "cu_seqlens": cu})
+    side = None
+    if world == 1 and not args.no_side and args.variant == "forced":
+        # the 32K shapes beside the headline one, measured in the same run
+        side = {n: side_workload(n, moba, dev, burst) for n in SIDE_WORKLOADS if n != w.name}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -957,6 +1030,7 @@ def main():
         "attn_kernels_frac_of_burst": attn_tflops / burst,
         "parity": parity,
         "input_sha256": hashes,
+        "side_workloads": side,
     }
     print(json.dumps(line), flush=True)
     if world > 1:
