@@ -14,11 +14,12 @@
 //
 // Two launches, both SIMT (a query row against its keys is a matrix-vector
 // product: HBM-bound, no tensor-core shape):
-//   decode_gate_kernel  one CTA per (query, head): threads score blocks
-//                       i = tid, tid + 128, ... (q in shared memory, the block
-//                       mean by 16-byte loads) into sorted lists, each warp
-//                       picks its k-1 best by rounds of warp arg-max, one
-//                       thread merges the warps' lists;
+//   decode_gate_kernel  one CTA per (query, head), 8 warps: a warp reads a
+//                       block mean with one coalesced 16-bytes-per-lane load,
+//                       reduces the dot product with q by shuffles, and the
+//                       lane owning the block keeps it in a sorted list; each
+//                       warp picks its k-1 best by rounds of warp arg-max,
+//                       and warp 0 merges the warps' lists the same way;
 //   decode_attn_kernel  split-K over the chosen keys: one CTA per (query,
 //                       q head, chosen block, chunk of <= 512 keys) keeps an
 //                       online softmax (m, l, o) per group of lanes that share
@@ -34,7 +35,7 @@
 namespace moba {
 namespace {
 
-constexpr int kGateWarps = 4;
+constexpr int kGateWarps = 8;
 constexpr int kAttnThreads = 256;
 constexpr int kAttnWarps = kAttnThreads / 32;
 
@@ -113,16 +114,35 @@ decode_gate_kernel(Dims dm, const T* __restrict__ q, const float* __restrict__ k
     ts[j] = -INFINITY;
     ti[j] = INT_MAX;
   }
-  const float4* qv = reinterpret_cast<const float4*>(qs);
-  for (int i = tid; i < c; i += kGateWarps * 32) {
-    const float4* kb = reinterpret_cast<const float4*>(kbar + (((int64_t)r * dm.nb + i) * dm.Hkv + g) * D);
-    float acc = 0.f;
-#pragma unroll 8
-    for (int x4 = 0; x4 < D / 4; ++x4) {
-      const float4 a = __ldg(kb + x4), b = qv[x4];
-      acc = fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
+  // Warp-cooperative scores: LPB lanes read one block mean together (16
+  // bytes each, one coalesced read of the block's d values), the dot product
+  // is reduced over those lanes, and one of them (by step) keeps the score
+  // in its sorted list. GU steps' loads are in flight together.
+  constexpr int LPB = D / 4;     // lanes per block mean
+  constexpr int BPS = 32 / LPB;  // block means a warp reads per step
+  constexpr int GU = 8;
+  const int grp_i = lane / LPB, sub = lane % LPB;
+  const float4 qv = reinterpret_cast<const float4*>(qs)[sub];
+  const int stride = kGateWarps * BPS;
+  const int nsteps = (c + stride - 1) / stride;
+  for (int s0 = 0; s0 < nsteps; s0 += GU) {
+    float4 kv[GU];
+#pragma unroll
+    for (int u = 0; u < GU; ++u) {
+      const int i = (s0 + u) * stride + warp * BPS + grp_i;
+      kv[u] = i < c ? __ldg(reinterpret_cast<const float4*>(
+                              kbar + (((int64_t)r * dm.nb + i) * dm.Hkv + g) * D) + sub)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    insert<KM>(ts, ti, acc, i);
+#pragma unroll
+    for (int u = 0; u < GU; ++u) {
+      float acc = fmaf(kv[u].w, qv.w, fmaf(kv[u].z, qv.z, fmaf(kv[u].y, qv.y, kv[u].x * qv.x)));
+#pragma unroll
+      for (int off = LPB / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      const int st = s0 + u;
+      const int i = st * stride + warp * BPS + grp_i;
+      if (i < c && sub == st % LPB) insert<KM>(ts, ti, acc, i);
+    }
   }
   // each warp: k-1 rounds of arg-max over the heads of its 32 sorted lists
   const int need = dm.topk - 1, hsel = min(need, c);
@@ -158,17 +178,52 @@ decode_gate_kernel(Dims dm, const T* __restrict__ q, const float* __restrict__ k
     }
   }
   __syncthreads();
-  if (tid != 0) return;
-  // the warps' lists into one: the k-1 best of all blocks
+  if (warp != 0) return;
+  // the warps' lists into one, by warp 0: each lane holds up to KC of the
+  // candidates in a sorted list, then k-1 rounds of warp arg-max
+  constexpr int KC = (kGateWarps * KM + 31) / 32;
+  float cs[KC];
+  int ci[KC];
+#pragma unroll
+  for (int j = 0; j < KC; ++j) {
+    cs[j] = -INFINITY;
+    ci[j] = INT_MAX;
+  }
+  for (int e = lane; e < kGateWarps * need; e += 32) insert<KC>(cs, ci, ws[e / need][e % need], wi[e / need][e % need]);
   float fs[KM];
   int fi[KM];
 #pragma unroll
-  for (int j = 0; j < KM; ++j) {
-    fs[j] = -INFINITY;
-    fi[j] = INT_MAX;
+  for (int rr = 0; rr < KM; ++rr) {
+    fs[rr] = -INFINITY;
+    fi[rr] = INT_MAX;
+    if (rr < need) {
+      float bs = cs[0];
+      int bi = ci[0], owner = lane;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        const int oo = __shfl_xor_sync(0xffffffffu, owner, off);
+        if (better(os, oi, bs, bi)) {
+          bs = os;
+          bi = oi;
+          owner = oo;
+        }
+      }
+      if (owner == lane) {
+#pragma unroll
+        for (int j = 0; j + 1 < KC; ++j) {
+          cs[j] = cs[j + 1];
+          ci[j] = ci[j + 1];
+        }
+        cs[KC - 1] = -INFINITY;
+        ci[KC - 1] = INT_MAX;
+      }
+      fs[rr] = bs;
+      fi[rr] = bi;
+    }
   }
-  for (int w = 0; w < kGateWarps; ++w)
-    for (int rr = 0; rr < need; ++rr) insert<KM>(fs, fi, ws[w][rr], wi[w][rr]);
+  if (lane != 0) return;
   int sel[KM];
 #pragma unroll
   for (int j = 0; j < KM; ++j) sel[j] = j < hsel ? fi[j] : INT_MAX;
