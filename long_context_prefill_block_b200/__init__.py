@@ -429,7 +429,7 @@ def dense_causal_forward(q, k, v, cu_seqlens, max_seqlen=None, return_lse: bool 
 
 
 def moba_selftest_bounded_wait(device=None) -> int:
-    """Run the bounded-wait self-test kernel; returns the kernel's verdict
+    """Run the bounded-wait self-test kernel; returns the kernel's result code
     (2 = the wait gave up as it must). Read moba_device_status() afterwards."""
     fn = lib().moba_selftest_bounded_wait
     fn.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
